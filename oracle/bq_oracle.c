@@ -1,0 +1,226 @@
+/*
+ * bq_oracle.c - plain CPU reference (see bq_oracle.h for what it follows).
+ *
+ * TEST INFRASTRUCTURE ONLY: used by tests/, the package smoke check and the
+ * benchmark's CPU-baseline leg; never by the library path.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (see oracle/build.py).  The code is a direct transcription of the method's
+ * definitions, one element at a time, with no blocking, vectorisation or
+ * reordering of the arithmetic.
+ */
+#include "bq_oracle.h"
+
+#include <math.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- types -- */
+
+static float bits_to_f32(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t f32_to_bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* IEEE binary16 -> binary32, exact (every binary16 value is a binary32 value). */
+float bqo_f16_to_f32(uint16_t h)
+{
+    int sign = h >> 15;
+    int e = (h >> 10) & 31;
+    int m = h & 1023;
+    float v;
+    if (e == 0)
+        v = ldexpf((float)m, -24);                 /* zero or subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexpf((float)(m + 1024), e - 25);     /* (1024 + m) * 2^(e - 15 - 10) */
+    return sign ? -v : v;
+}
+
+/* bfloat16 is the top half of a binary32. */
+float bqo_bf16_to_f32(uint16_t h) { return bits_to_f32((uint32_t)h << 16); }
+
+/* binary32 -> bfloat16, round to nearest, ties to even. */
+uint16_t bqo_f32_to_bf16(float f)
+{
+    uint32_t u = f32_to_bits(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u)           /* NaN: keep it a quiet NaN */
+        return (uint16_t)((u >> 16) | 0x40u);
+    uint32_t lower = u & 0xffffu;
+    uint32_t upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1;                                /* carries into the exponent */
+    return (uint16_t)upper;
+}
+
+/* binary32 -> binary16, round to nearest, ties to even. */
+uint16_t bqo_f32_to_f16(float f)
+{
+    uint32_t u = f32_to_bits(f);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t a = u & 0x7fffffffu;
+    if (a > 0x7f800000u)
+        return (uint16_t)(sign | 0x7e00u);         /* NaN */
+    if (a >= 0x477ff000u)                          /* >= 65520: rounds to infinity */
+        return (uint16_t)(sign | 0x7c00u);
+    if (a < 0x38800000u) {                         /* below 2^-14: subnormal range */
+        /* the result is round(|f| * 2^24) units of 2^-24; the product is exact
+         * in double and nearbyint rounds ties to even */
+        double units = nearbyint((double)fabsf(f) * 16777216.0);
+        return (uint16_t)(sign | (uint16_t)units); /* 1024 is the smallest normal */
+    }
+    /* normal: rebias the exponent (127 -> 15) and drop 13 mantissa bits */
+    uint32_t h = (a - 0x38000000u) >> 13;
+    uint32_t rem = a & 0x1fffu;
+    if (rem > 0x1000u || (rem == 0x1000u && (h & 1u)))
+        h += 1;
+    return (uint16_t)(sign | h);
+}
+
+static float load_elem(const void *x, int dtype, int64_t i)
+{
+    switch (dtype) {
+    case BQO_F32:  return ((const float *)x)[i];
+    case BQO_F16:  return bqo_f16_to_f32(((const uint16_t *)x)[i]);
+    default:       return bqo_bf16_to_f32(((const uint16_t *)x)[i]);
+    }
+}
+
+static void store_elem(void *y, int dtype, int64_t i, float v)
+{
+    switch (dtype) {
+    case BQO_F32:  ((float *)y)[i] = v; break;
+    case BQO_F16:  ((uint16_t *)y)[i] = bqo_f32_to_f16(v); break;
+    default:       ((uint16_t *)y)[i] = bqo_f32_to_bf16(v); break;
+    }
+}
+
+static int valid_dtype(int d) { return d == BQO_F32 || d == BQO_F16 || d == BQO_BF16; }
+
+static int valid_blocksize(int bs)
+{
+    /* bitsandbytes PR #2052: every block size from 32 through 4096 */
+    return bs >= 32 && bs <= 4096 && (bs & (bs - 1)) == 0;
+}
+
+/* ------------------------------------------------------ nearest code ---- */
+
+/*
+ * Nearest-code search as the plain definition: the distance to entry j is
+ * |RN(xn - code[j])| in binary32; the smallest distance wins and, on equal
+ * distances, the lowest index wins (strict "<" while scanning upwards).
+ */
+int bqo_nearest_code(float xn, const float *code, int entries)
+{
+    int idx = 0;
+    float best = fabsf(xn - code[0]);
+    for (int j = 1; j < entries; ++j) {
+        float d = fabsf(xn - code[j]);
+        if (d < best) {
+            best = d;
+            idx = j;
+        }
+    }
+    return idx;
+}
+
+/* ---------------------------------------------------------- quantize ---- */
+
+int bqo_quantize_blockwise(const void *x, int dtype, int64_t n, int blocksize,
+                           const float *code, int entries,
+                           float *absmax, uint8_t *out)
+{
+    if (n < 0 || !valid_dtype(dtype) || !valid_blocksize(blocksize) ||
+        (entries != 16 && entries != 256))
+        return -1;
+    if (n == 0)
+        return 0;
+    int64_t nb = (n + blocksize - 1) / blocksize;
+    int64_t out_bytes = entries == 16 ? (n + 1) / 2 : n;
+    memset(out, 0, (size_t)out_bytes);
+
+    for (int64_t b = 0; b < nb; ++b) {
+        int64_t lo = b * blocksize;
+        int64_t hi = lo + blocksize < n ? lo + blocksize : n;
+
+        /* step 1: absmax over the block's valid elements */
+        float A = 0.0f;
+        for (int64_t i = lo; i < hi; ++i)
+            A = fmaxf(A, fabsf(load_elem(x, dtype, i)));
+        absmax[b] = A;
+
+        /* step 2: normalise by IEEE division, search the codebook, pack */
+        for (int64_t i = lo; i < hi; ++i) {
+            float v = load_elem(x, dtype, i);
+            float xn = (A == 0.0f) ? 0.0f : v / A;
+            int idx = bqo_nearest_code(xn, code, entries);
+            if (entries == 16) {
+                if ((i & 1) == 0)
+                    out[i >> 1] |= (uint8_t)(idx << 4);   /* element 2i: high nibble */
+                else
+                    out[i >> 1] |= (uint8_t)idx;          /* element 2i+1: low nibble */
+            } else {
+                out[i] = (uint8_t)idx;
+            }
+        }
+    }
+    return 0;
+}
+
+/* -------------------------------------------------------- dequantize ---- */
+
+int bqo_dequantize_blockwise(const uint8_t *q, const float *absmax, int64_t n,
+                             int blocksize, const float *code, int entries,
+                             void *y, int ydtype)
+{
+    if (n < 0 || !valid_dtype(ydtype) || !valid_blocksize(blocksize) ||
+        (entries != 16 && entries != 256))
+        return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        int idx;
+        if (entries == 16)
+            idx = (i & 1) ? (q[i >> 1] & 15) : (q[i >> 1] >> 4);
+        else
+            idx = q[i];
+        float v = code[idx] * absmax[i / blocksize];
+        store_elem(y, ydtype, i, v);
+    }
+    return 0;
+}
+
+/* -------------------------------------------------------------- GGUF ---- */
+
+static float block_scale(const uint8_t *blk)
+{
+    return bqo_f16_to_f32((uint16_t)(blk[0] | (blk[1] << 8)));
+}
+
+int bqo_dequant_q8_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 34 * k;
+        float d = block_scale(blk);
+        for (int j = 0; j < 32; ++j) {
+            int qv = (int)(int8_t)blk[2 + j];
+            store_elem(y, ydtype, 32 * k + j, d * (float)qv);
+        }
+    }
+    return 0;
+}
+
+int bqo_dequant_q4_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 18 * k;
+        float d = block_scale(blk);
+        for (int j = 0; j < 16; ++j) {
+            int lo = blk[2 + j] & 15;      /* shift 0: elements 0..15  */
+            int hi = blk[2 + j] >> 4;      /* shift 4: elements 16..31 */
+            store_elem(y, ydtype, 32 * k + j, d * (float)(lo - 8));
+            store_elem(y, ydtype, 32 * k + 16 + j, d * (float)(hi - 8));
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,73 @@
+/*
+ * bq_oracle.h - plain, slow, single-threaded CPU reference for blockwise
+ * codebook quantization / dequantization and GGUF Q8_0 / Q4_0 dequantization.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library path may include, link
+ * or call this code: only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg use it.  It shares no code, header, table or
+ * constant with the CUDA implementation.
+ *
+ * What it follows (page titles of the source material):
+ *  - "bitsandbytes PR #2052, Respect the current CUDA stream in blockwise
+ *    quantization", Summary and Correctness sections: blockwise quantization
+ *    with General8 (dynamic 8-bit), FP4 and NF4 maps, block sizes 32..4096,
+ *    full blocks and tails, FP16/BF16/FP32 inputs.
+ *  - "ComfyUI-GGUF PR #472, Cache device-side constants in dequant kernels",
+ *    Problem section (Q4_0 low nibble then high nibble, shift vector [0, 4])
+ *    and the Verification table (Q8_0 and Q4_0 rows).
+ *  - "Model-Optimizer PR #2448" review notes: lowest index wins on equal
+ *    error; fused multiply-add changes near-ties, so this file is compiled
+ *    with contraction off (-ffp-contract=off) and no fast-math.
+ *
+ * Every floating-point operation here is one IEEE-754 binary32 operation
+ * rounded to nearest-even, in source order.
+ */
+#ifndef BQ_ORACLE_H
+#define BQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type codes used by this oracle (its own numbering). */
+enum { BQO_F32 = 0, BQO_F16 = 1, BQO_BF16 = 2 };
+
+/* Exact widening and round-to-nearest-even narrowing. */
+float    bqo_f16_to_f32(uint16_t h);
+float    bqo_bf16_to_f32(uint16_t h);
+uint16_t bqo_f32_to_f16(float f);
+uint16_t bqo_f32_to_bf16(float f);
+
+/* Nearest codebook entry: argmin_j |RN(xn - code[j])|, lowest j on ties. */
+int bqo_nearest_code(float xn, const float *code, int entries);
+
+/*
+ * Blockwise absmax codebook quantization of x[0..n) (element type dtype).
+ * absmax[b] = max |x_i| over block b (the last block may be short).
+ * entries == 16: out has ceil(n/2) bytes, element 2i in the high nibble of
+ * byte i, element 2i+1 in the low nibble (0 when it does not exist).
+ * entries == 256: out has n bytes, one code per element.
+ * Returns 0 on success, -1 on a bad argument.
+ */
+int bqo_quantize_blockwise(const void *x, int dtype, int64_t n, int blocksize,
+                           const float *code, int entries,
+                           float *absmax, uint8_t *out);
+
+/* y_i = narrow(RN(code[idx_i] * absmax[i / blocksize])). */
+int bqo_dequantize_blockwise(const uint8_t *q, const float *absmax, int64_t n,
+                             int blocksize, const float *code, int entries,
+                             void *y, int ydtype);
+
+/* GGUF Q8_0: 34-byte blocks {fp16 d (little endian), int8 q[32]}. */
+int bqo_dequant_q8_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q4_0: 18-byte blocks {fp16 d, uint8 qs[16]};
+ * y[32k+j] = d*((qs[j] & 15) - 8), y[32k+16+j] = d*((qs[j] >> 4) - 8). */
+int bqo_dequant_q4_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
