@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark: quantize / dequantize HBM GB/s (input + output bytes) on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  1. blockwise quantize   bf16 n = 2^29 (1 GiB), NF4, blocksize 64
+     (N(0, 0.02) with 0.1% outliers from N(0, 0.4))
+  2. blockwise dequantize of the result back to bf16
+  3. GGUF Q8_0 dequant of a 4096 x 14336 matrix (1,835,008 blocks) to bf16
+  4. GGUF Q4_0 dequant of a 4096 x 14336 matrix to bf16
+value = (input + output bytes of the four kernels) / device time, in GB/s.
+Inputs (1 GiB) are larger than L2 (126 MB), so no flush is needed.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torch.distributed.run; every rank runs the same workload
+on its own GPU (weak scaling, no collective on the data path).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bq_inputs import codebooks, synth  # noqa: E402
+
+METRIC = "quantize/dequantize HBM GB/s (in+out bytes) and % of B200 HBM peak"
+N_LARGE = synth.LARGE_N
+BS = 64
+GGUF_BLOCKS = 4096 * 14336 // 32
+WORKLOAD = ("bf16 NF4 blocksize-64 quantize + dequantize of n=2^29 (1 GiB, N(0,0.02) + 0.1% "
+            "N(0,0.4) outliers), then GGUF Q8_0 and Q4_0 dequant of a 4096x14336 matrix to bf16")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--n", type=int, default=N_LARGE, help="elements of the quantize input")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
+                    default="all", help="run one kernel per step (profiling aid)")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ bytes --
+
+def quant_bytes(n, bs, elem=2):
+    """Algorithmic bytes of one quantize (or dequantize) launch: n*elem input
+    (output), ceil(n/2) packed codes, 4 bytes of absmax per block."""
+    return n * elem + (n + 1) // 2 + 4 * ((n + bs - 1) // bs)
+
+
+def gguf_bytes(nblk, block_bytes, out_elem=2):
+    return nblk * block_bytes + 32 * nblk * out_elem
+
+
+def step_bytes(n, nblk, only="all"):
+    parts = {"quantize": quant_bytes(n, BS), "dequantize": quant_bytes(n, BS),
+             "q8_0": gguf_bytes(nblk, 34), "q4_0": gguf_bytes(nblk, 18)}
+    if only != "all":
+        return {only: parts[only]}
+    return parts
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.lines = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:  # pragma: no cover - nvidia-smi missing
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ peaks --
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dequantization_bq_quantize_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when the kernel sources changed since those counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("csrc_sha") != csrc_digest():
+        return None
+    v = t.get("kernels", {}).get(kernel)
+    return None if v is None else float(v["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------- distributed ----
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    if args.gpus != world and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- reference ---
+
+def run_reference(args, rank, world):
+    """The oracle (plain single-threaded C, driven over disjoint block ranges
+    on every host core) on a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle.host_threads()
+    n_s = 1 << 25
+    nblk_s = 1 << 16
+    x, _ = synth.large_outliers(n=n_s)
+    xb = synth.to_numpy_bits(x)
+    nf4 = codebooks.nf4()
+    q8 = synth.gguf_blocks(nblk_s, "q8_0", seed=4)
+    q4 = synth.gguf_blocks(nblk_s, "q4_0", seed=5)
+    byts = sum(step_bytes(n_s, nblk_s).values())
+
+    def one_step():
+        a, q = oracle.quantize_blockwise_threaded(xb, "bf16", BS, nf4, threads)
+        oracle.dequantize_blockwise_threaded(q, a, n_s, BS, nf4, "bf16", threads)
+        oracle.dequant_q8_0(q8, "bf16")
+        oracle.dequant_q4_0(q4, "bf16")
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = byts / dt / 1e9
+    sample = (f"per step: quantize+dequantize of the first 2^25 elements of the bf16 workload "
+              f"and Q8_0/Q4_0 dequant of 2^16 blocks each; {threads} host threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_elements": n_s, "sample_gguf_blocks": nblk_s},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(n, nblk, x_cpu):
+    """Oracle timed on the host cores on a bounded sample (~10-30 s of CPU work)."""
+    import oracle
+    threads = oracle.host_threads()
+    n_s = min(n, 1 << 26)
+    nblk_s = min(nblk, 1 << 18)
+    xb = synth.to_numpy_bits(x_cpu[:n_s])
+    nf4 = codebooks.nf4()
+    q8 = synth.gguf_blocks(nblk_s, "q8_0", seed=4)
+    q4 = synth.gguf_blocks(nblk_s, "q4_0", seed=5)
+    t0 = time.perf_counter()
+    a, q = oracle.quantize_blockwise_threaded(xb, "bf16", BS, nf4, threads)
+    oracle.dequantize_blockwise_threaded(q, a, n_s, BS, nf4, "bf16", threads)
+    oracle.dequant_q8_0(q8, "bf16")
+    oracle.dequant_q4_0(q4, "bf16")
+    dt = time.perf_counter() - t0
+    byts = sum(step_bytes(n_s, nblk_s).values())
+    return {"value": round(byts / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": (f"quantize+dequantize of the first 2^26 elements of the step's bf16 input "
+                       f"({threads} threads over disjoint block ranges) and single-threaded "
+                       f"Q8_0/Q4_0 dequant of 2^18 blocks each; {dt:.2f} s wall")}
+
+
+# -------------------------------------------------------------------- ours --
+
+class Workload:
+    def __init__(self, n, rank, device):
+        import dequantization_bq_quantize_b200 as bq
+        self.bq = bq
+        bq.lib()
+        self.n = n
+        self.nb = (n + BS - 1) // BS
+        self.nblk = GGUF_BLOCKS
+        x_cpu, self.outliers = synth.large_outliers(n=n, seed=3 + 1000 * rank)
+        self.x_cpu = x_cpu
+        self.x = x_cpu.to(device)
+        self.code = torch.from_numpy(codebooks.nf4()).to(device)
+        self.absmax = torch.empty(self.nb, dtype=torch.float32, device=device)
+        self.q = torch.empty((n + 1) // 2, dtype=torch.uint8, device=device)
+        self.y = torch.empty(n, dtype=torch.bfloat16, device=device)
+        q8 = synth.gguf_blocks(self.nblk, "q8_0", seed=4 + 1000 * rank)
+        q4 = synth.gguf_blocks(self.nblk, "q4_0", seed=5 + 1000 * rank)
+        self.q8_cpu = torch.from_numpy(q8.reshape(-1))
+        self.q4_cpu = torch.from_numpy(q4.reshape(-1))
+        self.q8 = self.q8_cpu.to(device)
+        self.q4 = self.q4_cpu.to(device)
+        self.y8 = torch.empty(32 * self.nblk, dtype=torch.bfloat16, device=device)
+        self.y4 = torch.empty(32 * self.nblk, dtype=torch.bfloat16, device=device)
+
+    def kernels(self, only):
+        bq = self.bq
+        names = ["quantize", "dequantize", "q8_0", "q4_0"] if only == "all" else [only]
+        return names
+
+    def launch(self, name, stream):
+        bq = self.bq
+        if name == "quantize":
+            st = bq.bq_quantize_blockwise(self.x.data_ptr(), bq.BQ_BF16, self.n, BS,
+                                          self.code.data_ptr(), 16, self.absmax.data_ptr(),
+                                          self.q.data_ptr(), stream)
+        elif name == "dequantize":
+            st = bq.bq_dequantize_blockwise(self.q.data_ptr(), self.absmax.data_ptr(), self.n, BS,
+                                            self.code.data_ptr(), 16, self.y.data_ptr(),
+                                            bq.BQ_BF16, stream)
+        elif name == "q8_0":
+            st = bq.bq_dequant_q8_0(self.q8.data_ptr(), self.nblk, self.y8.data_ptr(), bq.BQ_BF16,
+                                    stream)
+        else:
+            st = bq.bq_dequant_q4_0(self.q4.data_ptr(), self.nblk, self.y4.data_ptr(), bq.BQ_BF16,
+                                    stream)
+        if st != bq.BQ_OK:
+            raise RuntimeError(f"{name}: {bq.bq_status_string(st)} {bq.bq_last_cuda_error()}")
+
+
+def run_ours(args, rank, world, local):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = Workload(args.n, rank, dev)
+    names = w.kernels(args.only)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    byts = step_bytes(w.n, w.nblk, args.only)
+    step_total = sum(byts.values())
+
+    for _ in range(args.warmup):
+        for k in names:
+            w.launch(k, sh)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    time.sleep(0.3)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        for i, k in enumerate(names):
+            w.launch(k, sh)
+            ev[s][i + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    total_ms = ev[0][0].elapsed_time(ev[-1][-1])
+    per_kernel = {k: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)]
+                  for i, k in enumerate(names)}
+    max_ms = max_over_ranks(total_ms, world)
+    ms_per_step = max_ms / args.steps
+    value = step_total * world / (ms_per_step / 1e3) / 1e9
+
+    # ---- end to end: host buffers in, results back to the host, every step
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, names, stream, sh, byts, world)
+
+    peak, peak_kind = measured_peaks()
+    kern = {}
+    for k in names:
+        ms = statistics.mean(per_kernel[k])
+        gbs = byts[k] / (ms / 1e3) / 1e9
+        kern[k] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                   "bytes": byts[k]}
+    dom = "quantize" if "quantize" in kern else names[0]
+    kname = {"quantize": "quantize_kernel<bf16,nf4,bs64>", "dequantize":
+             "dequant_kernel<nf4,bf16>", "q8_0": "gguf_kernel<q8_0,bf16>",
+             "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
+    roof = {"bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak, "unit": "GB/s",
+            "frac": kern[dom]["frac"], "traffic": recorded_traffic(kname),
+            "kernel": kname, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w.n, w.nblk, w.x_cpu)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "n": w.n, "blocksize": BS, "codebook": "nf4",
+                       "gguf_blocks": w.nblk, "outliers": w.outliers, "kernels": names,
+                       "l2": "inputs larger than L2 (126 MB); no flush",
+                       "parallelism": f"dp{world} (independent shards, no collective)"},
+            "roofline": roof,
+            "kernels": kern,
+            "pct_of_nominal_8tbs": {k: round(v["gbs"] / 8000.0, 4) for k, v in kern.items()},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": len(names) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, names, stream, sh, byts, world):
+    """Same step through the public API with host buffers: pinned host->device
+    copy of the step's inputs and device->host copy of its results, inside the
+    timed region, every step."""
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    xh = pin(w.x_cpu)
+    q8h, q4h = pin(w.q8_cpu), pin(w.q4_cpu)
+    outs = {"quantize": [w.absmax, w.q], "dequantize": [w.y], "q8_0": [w.y8], "q4_0": [w.y4]}
+    ins = {"quantize": [(w.x, xh)], "dequantize": [], "q8_0": [(w.q8, q8h)],
+           "q4_0": [(w.q4, q4h)]}
+    hosts = {k: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs[k]]
+             for k in names}
+    h2d = sum(h.numel() * h.element_size() for k in names for _, h in ins[k])
+    d2h = sum(t.numel() * t.element_size() for k in names for t in outs[k])
+    steps = max(1, min(args.steps, 5))
+
+    def one():
+        for k in names:
+            for d, h in ins[k]:
+                d.copy_(h, non_blocking=True)
+            w.launch(k, sh)
+            for d, h in zip(outs[k], hosts[k]):
+                h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    total = sum(byts.values()) * world
+    return {"value": round(total / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "steps": steps}
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

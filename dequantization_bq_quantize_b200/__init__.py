@@ -1,0 +1,204 @@
+"""Blockwise codebook quantization / dequantization and GGUF Q8_0 / Q4_0
+dequantization on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libbq.so`` (C ABI in ``include/bq.h``).  Every
+step of the computation runs in the library's CUDA kernels; this module only
+marshals arguments.  torch is used for device memory and streams.  There is no
+CPU fallback: if ``libbq.so`` is missing, every call raises.
+
+Raw ABI functions keep the C names (``bq_quantize_blockwise`` ...) and take
+integer device addresses.  The torch helpers (``quantize_blockwise`` ...) take
+CUDA tensors, allocate missing outputs with torch, and launch on the current
+torch stream unless a stream is given.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbq.so")
+
+BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_CUDA = 0, 1, 2, 3
+BQ_F32, BQ_F16, BQ_BF16 = 0, 1, 2
+
+EXPORTED = (
+    "bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
+    "bq_dequant_q4_0", "bq_status_string", "bq_last_cuda_error", "bq_device_fault",
+    "bq_abi_version",
+)
+
+_lib = None
+
+
+class BQError(RuntimeError):
+    """A bq entry point returned a status other than BQ_OK."""
+
+    def __init__(self, fn, status, detail):
+        self.status = status
+        super().__init__(f"{fn}: {detail}")
+
+
+def lib():
+    """The loaded libbq.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m dequantization_bq_quantize_b200._build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        L.bq_quantize_blockwise.argtypes = [vp, i32, i64, i32, vp, i32, vp, vp, vp]
+        L.bq_dequantize_blockwise.argtypes = [vp, vp, i64, i32, vp, i32, vp, i32, vp]
+        L.bq_dequant_q8_0.argtypes = [vp, i64, vp, i32, vp]
+        L.bq_dequant_q4_0.argtypes = [vp, i64, vp, i32, vp]
+        for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
+                  "bq_dequant_q4_0", "bq_device_fault"):
+            getattr(L, f).restype = ctypes.c_int
+        L.bq_status_string.argtypes = [ctypes.c_int]
+        L.bq_status_string.restype = ctypes.c_char_p
+        L.bq_last_cuda_error.argtypes = []
+        L.bq_last_cuda_error.restype = ctypes.c_char_p
+        L.bq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
+        L.bq_abi_version.argtypes = []
+        L.bq_abi_version.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def build(force=False):
+    """Compile libbq.so in-tree (nvcc, sm_100a)."""
+    from . import _build
+    return _build.build(force=force)
+
+
+# ------------------------------------------------------------ raw C ABI ----
+
+def bq_quantize_blockwise(x, x_dtype, n, blocksize, code, code_entries, absmax, out, stream):
+    return lib().bq_quantize_blockwise(x, x_dtype, n, blocksize, code, code_entries, absmax, out,
+                                       stream)
+
+
+def bq_dequantize_blockwise(q, absmax, n, blocksize, code, code_entries, y, y_dtype, stream):
+    return lib().bq_dequantize_blockwise(q, absmax, n, blocksize, code, code_entries, y, y_dtype,
+                                         stream)
+
+
+def bq_dequant_q8_0(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q8_0(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q4_0(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q4_0(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_status_string(status):
+    return lib().bq_status_string(status).decode()
+
+
+def bq_last_cuda_error():
+    return lib().bq_last_cuda_error().decode()
+
+
+def bq_device_fault(reset=True):
+    """Read (and by default clear) the device fault word; synchronizes."""
+    v = ctypes.c_uint32(0)
+    _check("bq_device_fault", lib().bq_device_fault(ctypes.byref(v), 1 if reset else 0))
+    return v.value
+
+
+def bq_abi_version():
+    return lib().bq_abi_version()
+
+
+def _check(fn, status):
+    if status != BQ_OK:
+        detail = bq_status_string(status)
+        extra = bq_last_cuda_error()
+        raise BQError(fn, status, f"{detail} ({extra})" if extra else detail)
+
+
+# --------------------------------------------------------- torch helpers ----
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(dt):
+    torch = _torch()
+    return {torch.float32: BQ_F32, torch.float16: BQ_F16, torch.bfloat16: BQ_BF16}[dt]
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need_cuda(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def code_bytes(n, entries):
+    """Bytes of packed codes for n elements (two per byte for 16 entries)."""
+    return (n + 1) // 2 if entries == 16 else n
+
+
+def quantize_blockwise(x, code, blocksize, absmax=None, out=None, stream=None):
+    """Quantize the CUDA tensor x (fp32/fp16/bf16, any shape, flattened).
+
+    code: CUDA float32 tensor of 16 or 256 sorted entries.
+    Returns (absmax float32[ceil(n/blocksize)], packed codes uint8)."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    _need_cuda(code, "code")
+    n = x.numel()
+    entries = code.numel()
+    nb = (n + blocksize - 1) // blocksize
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=x.device)
+    if out is None:
+        out = torch.empty(code_bytes(n, entries), dtype=torch.uint8, device=x.device)
+    _check("bq_quantize_blockwise", bq_quantize_blockwise(
+        x.data_ptr(), _dtype_code(x.dtype), n, blocksize, code.data_ptr(), entries,
+        absmax.data_ptr(), out.data_ptr(), _stream_handle(stream)))
+    return absmax, out
+
+
+def dequantize_blockwise(q, absmax, n, blocksize, code, dtype=None, out=None, stream=None):
+    """Inverse of quantize_blockwise: n values of ``dtype`` (default bf16)."""
+    torch = _torch()
+    _need_cuda(q, "q")
+    _need_cuda(absmax, "absmax")
+    _need_cuda(code, "code")
+    if out is None:
+        out = torch.empty(n, dtype=dtype or torch.bfloat16, device=q.device)
+    _check("bq_dequantize_blockwise", bq_dequantize_blockwise(
+        q.data_ptr(), absmax.data_ptr(), n, blocksize, code.data_ptr(), code.numel(),
+        out.data_ptr(), _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+def _gguf(fn, bbytes, blocks, dtype, out, stream):
+    torch = _torch()
+    _need_cuda(blocks, "blocks")
+    nblk = blocks.numel() // bbytes
+    if out is None:
+        out = torch.empty(32 * nblk, dtype=dtype or torch.bfloat16, device=blocks.device)
+    _check(fn.__name__, fn(blocks.data_ptr(), nblk, out.data_ptr(), _dtype_code(out.dtype),
+                           _stream_handle(stream)))
+    return out
+
+
+def dequant_q8_0(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q8_0 blocks (uint8 CUDA tensor of n_blocks*34 bytes) -> 32*n_blocks values."""
+    return _gguf(bq_dequant_q8_0, 34, blocks, dtype, out, stream)
+
+
+def dequant_q4_0(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q4_0 blocks (uint8 CUDA tensor of n_blocks*18 bytes) -> 32*n_blocks values."""
+    return _gguf(bq_dequant_q4_0, 18, blocks, dtype, out, stream)

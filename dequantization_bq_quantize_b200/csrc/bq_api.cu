@@ -1,0 +1,360 @@
+// bq_api.cu - the C ABI of libbq.so (declared in include/bq.h): host-side
+// validation, launch-configuration choice, TMA descriptor encoding, error
+// reporting.  All kernels live in this one translation unit.
+#include "bq.h"
+
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bq_dequant.cuh"
+#include "bq_gguf.cuh"
+#include "bq_quantize.cuh"
+
+static_assert(int(BQ_F32) == int(bq::kF32) && int(BQ_F16) == int(bq::kF16) &&
+                  int(BQ_BF16) == int(bq::kBF16),
+              "dtype codes must match");
+
+namespace {
+
+thread_local std::string t_err;
+
+bq_status cuda_fail(cudaError_t e, const char* what) {
+  t_err = std::string(what) + ": " + cudaGetErrorString(e);
+  return BQ_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+
+// Per-device facts, read once per device.
+struct DevInfo {
+  int sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+bq_status current_device(int* dev, DevInfo* info) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) {
+    t_err = "device ordinal out of range";
+    return BQ_ERR_UNSUPPORTED;
+  }
+  cudaError_t ie = cudaSuccess;
+  std::call_once(g_dev_once[*dev], [&] {
+    ie = cudaDeviceGetAttribute(&g_dev[*dev].sms, cudaDevAttrMultiProcessorCount, *dev);
+  });
+  if (ie != cudaSuccess) return cuda_fail(ie, "cudaDeviceGetAttribute");
+  if (g_dev[*dev].sms <= 0) {
+    t_err = "device attributes unavailable";
+    return BQ_ERR_CUDA;
+  }
+  *info = g_dev[*dev];
+  return BQ_OK;
+}
+
+// Per (kernel, device) one-time set-up: dynamic shared memory limit and the
+// number of resident CTAs per SM.
+struct KernelSlot {
+  std::once_flag once[kMaxDevices];
+  int occ[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+};
+
+template <typename K>
+bq_status kernel_occupancy(KernelSlot& slot, K kernel, int dev, int threads, size_t smem,
+                           int* occ) {
+  std::call_once(slot.once[dev], [&] {
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    int o = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kernel, threads, smem);
+    slot.err[dev] = e;
+    slot.occ[dev] = o;
+  });
+  if (slot.err[dev] != cudaSuccess) return cuda_fail(slot.err[dev], "kernel set-up");
+  *occ = slot.occ[dev] > 0 ? slot.occ[dev] : 1;
+  return BQ_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, fetched through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool valid_dtype(int d) { return d == BQ_F32 || d == BQ_F16 || d == BQ_BF16; }
+int elem_bytes(int d) { return d == BQ_F32 ? 4 : 2; }
+bool valid_blocksize(int32_t bs) { return bs >= 32 && bs <= 4096 && (bs & (bs - 1)) == 0; }
+int log2i(int32_t v) { int l = 0; while ((1 << l) < v) ++l; return l; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ------------------------------------------------------------- quantize ---
+
+template <int DT, int E, int TPB>
+bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev, int sms,
+                          cudaStream_t stream) {
+  static KernelSlot slot;
+  auto kernel = bq::quantize_kernel<DT, E, TPB>;
+  constexpr size_t smem = bq::qsmem_bytes<E>();
+  int occ = 1;
+  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kQThreads, smem, &occ);
+  if (s != BQ_OK) return s;
+  constexpr int BPT = bq::kQConsumers / TPB;
+  const int64_t gen_blocks = p.nb - p.full_tiles * BPT;
+  int64_t want = p.full_tiles;
+  const int64_t want_gen = (gen_blocks + bq::kQConsumers / 32 - 1) / (bq::kQConsumers / 32);
+  if (want_gen > want) want = want_gen;
+  if (want < 1) want = 1;
+  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  kernel<<<grid, bq::kQThreads, smem, stream>>>(map, p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "quantize launch");
+}
+
+template <int DT, int E>
+bq_status dispatch_quantize_bs(const bq::QParams& p, const CUtensorMap& map, int dev, int sms,
+                               cudaStream_t stream) {
+  constexpr int EPT = 64 / bq::ElemBytes<DT>::value;
+  switch (p.bs / EPT) {
+    case 1: if constexpr (EPT == 32) return launch_quantize<DT, E, 1>(p, map, dev, sms, stream); break;
+    case 2: return launch_quantize<DT, E, 2>(p, map, dev, sms, stream);
+    case 4: return launch_quantize<DT, E, 4>(p, map, dev, sms, stream);
+    case 8: return launch_quantize<DT, E, 8>(p, map, dev, sms, stream);
+    case 16: return launch_quantize<DT, E, 16>(p, map, dev, sms, stream);
+    case 32: return launch_quantize<DT, E, 32>(p, map, dev, sms, stream);
+    case 64: return launch_quantize<DT, E, 64>(p, map, dev, sms, stream);
+    case 128: return launch_quantize<DT, E, 128>(p, map, dev, sms, stream);
+    case 256: if constexpr (EPT == 16) return launch_quantize<DT, E, 256>(p, map, dev, sms, stream); break;
+    default: break;
+  }
+  t_err = "no kernel for this blocksize";
+  return BQ_ERR_UNSUPPORTED;
+}
+
+template <int DT>
+bq_status dispatch_quantize(const bq::QParams& p, int entries, const CUtensorMap& map, int dev,
+                            int sms, cudaStream_t stream) {
+  if (entries == 16) return dispatch_quantize_bs<DT, 16>(p, map, dev, sms, stream);
+  return dispatch_quantize_bs<DT, 256>(p, map, dev, sms, stream);
+}
+
+// ----------------------------------------------------------- dequantize ---
+
+template <int E, int OT>
+bq_status launch_dequant(const bq::DParams& p, int dev, int sms, cudaStream_t stream) {
+  static KernelSlot slot;
+  auto kernel = bq::dequant_kernel<E, OT>;
+  int occ = 1;
+  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kDThreads, 0, &occ);
+  if (s != BQ_OK) return s;
+  const int64_t work = p.vec ? (p.nchunks + 3) / 4 + 1 : p.n;
+  int64_t want = (work + bq::kDThreads - 1) / bq::kDThreads;
+  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  kernel<<<static_cast<int>(want), bq::kDThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "dequantize launch");
+}
+
+template <int OT>
+bq_status dispatch_dequant(const bq::DParams& p, int entries, int dev, int sms, cudaStream_t st) {
+  if (entries == 16) return launch_dequant<16, OT>(p, dev, sms, st);
+  return launch_dequant<256, OT>(p, dev, sms, st);
+}
+
+// ----------------------------------------------------------------- GGUF ---
+
+template <int KIND, int OT>
+bq_status launch_gguf(const bq::GParams& p, int dev, int sms, cudaStream_t stream) {
+  static KernelSlot slot;
+  auto kernel = bq::gguf_kernel<KIND, OT>;
+  int occ = 1;
+  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kGThreads, 0, &occ);
+  if (s != BQ_OK) return s;
+  const int64_t groups = (p.n_blocks + bq::kGGroup - 1) / bq::kGGroup;
+  int64_t want = (groups + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
+  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  kernel<<<static_cast<int>(want), bq::kGThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "gguf dequant launch");
+}
+
+template <int KIND>
+bq_status gguf_entry(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                     cudaStream_t stream) {
+  t_err.clear();
+  if (n_blocks < 0 || !valid_dtype(y_dtype)) return BQ_ERR_INVALID_ARG;
+  if (n_blocks == 0) return BQ_OK;
+  if (n_blocks > (int64_t{1} << 52)) return BQ_ERR_INVALID_ARG;
+  if (!blocks || !y || !aligned(y, elem_bytes(y_dtype))) return BQ_ERR_INVALID_ARG;
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+  bq::GParams p;
+  p.blocks = static_cast<const uint8_t*>(blocks);
+  p.y = y;
+  p.n_blocks = n_blocks;
+  p.vec = aligned(blocks, 16) && aligned(y, 16);
+  switch (y_dtype) {
+    case BQ_F32: return launch_gguf<KIND, bq::kF32>(p, dev, info.sms, stream);
+    case BQ_F16: return launch_gguf<KIND, bq::kF16>(p, dev, info.sms, stream);
+    default: return launch_gguf<KIND, bq::kBF16>(p, dev, info.sms, stream);
+  }
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+
+extern "C" {
+
+bq_status bq_quantize_blockwise(const void* x, bq_dtype x_dtype, int64_t n, int32_t blocksize,
+                                const float* code, int32_t code_entries, float* absmax,
+                                uint8_t* out, cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(x_dtype) || !valid_blocksize(blocksize) ||
+      (code_entries != 16 && code_entries != 256))
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (n > (int64_t{1} << 50)) return BQ_ERR_INVALID_ARG;
+  const int eb = elem_bytes(x_dtype);
+  if (!x || !code || !absmax || !out || !aligned(x, eb) || !aligned(absmax, 4) || !aligned(code, 4))
+    return BQ_ERR_INVALID_ARG;
+
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+
+  bq::QParams p;
+  p.x = x;
+  p.n = n;
+  p.code = code;
+  p.absmax = absmax;
+  p.out = out;
+  p.bs = blocksize;
+  p.nb = (n + blocksize - 1) / blocksize;
+  p.full_tiles = 0;
+
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  const int64_t rows = n * eb / bq::kTileRows;             // whole 128-byte rows
+  const int64_t tiles = rows / bq::kTileRows;              // whole 16 KiB tiles
+  if (tiles > 0 && aligned(x, 16) && aligned(out, 16) && rows < (int64_t{1} << 31)) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+    if (enc) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(bq::kTileRows), static_cast<cuuint64_t>(rows)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(bq::kTileRows)};
+      cuuint32_t box[2] = {128, static_cast<cuuint32_t>(bq::kTileRows)};
+      cuuint32_t estr[2] = {1, 1};
+      CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x), dims, strides,
+                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r == CUDA_SUCCESS) p.full_tiles = tiles;
+    }
+  }
+
+  switch (x_dtype) {
+    case BQ_F32: return dispatch_quantize<bq::kF32>(p, code_entries, map, dev, info.sms, stream);
+    case BQ_F16: return dispatch_quantize<bq::kF16>(p, code_entries, map, dev, info.sms, stream);
+    default: return dispatch_quantize<bq::kBF16>(p, code_entries, map, dev, info.sms, stream);
+  }
+}
+
+bq_status bq_dequantize_blockwise(const uint8_t* q, const float* absmax, int64_t n,
+                                  int32_t blocksize, const float* code, int32_t code_entries,
+                                  void* y, bq_dtype y_dtype, cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(y_dtype) || !valid_blocksize(blocksize) ||
+      (code_entries != 16 && code_entries != 256))
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (n > (int64_t{1} << 50)) return BQ_ERR_INVALID_ARG;
+  if (!q || !absmax || !code || !y || !aligned(absmax, 4) || !aligned(code, 4) ||
+      !aligned(y, elem_bytes(y_dtype)))
+    return BQ_ERR_INVALID_ARG;
+
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+
+  bq::DParams p;
+  p.q = q;
+  p.absmax = absmax;
+  p.code = code;
+  p.y = y;
+  p.n = n;
+  p.bs_log2 = log2i(blocksize);
+  const int ce = 16 / elem_bytes(y_dtype);
+  const int qb = code_entries == 16 ? ce / 2 : ce;
+  p.vec = aligned(y, 16) && aligned(q, qb);
+  p.nchunks = p.vec ? n / ce : 0;
+  switch (y_dtype) {
+    case BQ_F32: return dispatch_dequant<bq::kF32>(p, code_entries, dev, info.sms, stream);
+    case BQ_F16: return dispatch_dequant<bq::kF16>(p, code_entries, dev, info.sms, stream);
+    default: return dispatch_dequant<bq::kBF16>(p, code_entries, dev, info.sms, stream);
+  }
+}
+
+bq_status bq_dequant_q8_0(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ8_0>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q4_0(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ4_0>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+const char* bq_status_string(bq_status s) {
+  switch (s) {
+    case BQ_OK: return "ok";
+    case BQ_ERR_INVALID_ARG: return "invalid argument";
+    case BQ_ERR_UNSUPPORTED: return "unsupported";
+    case BQ_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+const char* bq_last_cuda_error(void) { return t_err.c_str(); }
+
+bq_status bq_device_fault(uint32_t* fault, int32_t reset) {
+  t_err.clear();
+  if (!fault) return BQ_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, bq::g_fault, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the fault word");
+  *fault = v;
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(bq::g_fault, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the fault word");
+  }
+  return BQ_OK;
+}
+
+int32_t bq_abi_version(void) { return BQ_ABI_VERSION; }
+
+}  // extern "C"

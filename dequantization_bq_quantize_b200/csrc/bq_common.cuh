@@ -1,0 +1,159 @@
+// bq_common.cuh - shared device helpers for the bq kernels (sm_100a).
+//
+// Element widening, output narrowing, mbarrier / TMA wrappers written as
+// inline PTX, and the bounded wait used by every pipelined kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bq {
+
+// Element type codes, equal to the C ABI's bq_dtype values.
+enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
+
+template <int DT> struct ElemBytes { static constexpr int value = DT == kF32 ? 4 : 2; };
+
+// Fault word (one per device): bit 0 = a consumer gave up waiting for data,
+// bit 1 = a producer gave up waiting for a free stage.
+__device__ uint32_t g_fault;
+
+// A wait on an mbarrier gives up after this many nanoseconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------- widening --
+
+// Element j of a 16-bit-element vector held as 32-bit words (element 2i in the
+// low half of word i: little-endian order of the bytes in memory).
+template <int DT>
+__device__ __forceinline__ float widen_pair_elem(uint32_t w, int hi);
+
+template <>
+__device__ __forceinline__ float widen_pair_elem<kBF16>(uint32_t w, int hi) {
+  return __uint_as_float(hi ? (w & 0xffff0000u) : (w << 16));
+}
+
+template <>
+__device__ __forceinline__ float widen_pair_elem<kF16>(uint32_t w, int hi) {
+  return __half2float(__ushort_as_half((unsigned short)(hi ? (w >> 16) : (w & 0xffffu))));
+}
+
+// Scalar element load from global memory (any alignment of the element type).
+template <int DT>
+__device__ __forceinline__ float load_elem(const void* x, int64_t i) {
+  if constexpr (DT == kF32) {
+    return static_cast<const float*>(x)[i];
+  } else {
+    uint32_t h = static_cast<const unsigned short*>(x)[i];
+    return widen_pair_elem<DT>(h, 0);
+  }
+}
+
+// --------------------------------------------------------------- narrowing --
+
+// Round-to-nearest-even narrowing of two fp32 values into one 32-bit word
+// (first value in the low half).
+template <int OT>
+__device__ __forceinline__ uint32_t narrow2(float a, float b);
+
+template <>
+__device__ __forceinline__ uint32_t narrow2<kBF16>(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <>
+__device__ __forceinline__ uint32_t narrow2<kF16>(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int OT>
+__device__ __forceinline__ void store_elem(void* y, int64_t i, float v) {
+  if constexpr (OT == kF32) {
+    static_cast<float*>(y)[i] = v;
+  } else if constexpr (OT == kBF16) {
+    static_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
+  } else {
+    static_cast<__half*>(y)[i] = __float2half_rn(v);
+  }
+}
+
+// ------------------------------------------------------------ PTX wrappers --
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed; false if that
+// does not happen within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// 2-D tiled TMA load (no multicast) into this CTA's shared memory, completing
+// `bar`'s transaction count.  c0 is the inner (byte) coordinate.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32), id != 0.
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void record_fault(uint32_t bit) { atomicOr(&g_fault, bit); }
+
+}  // namespace bq

@@ -1,0 +1,151 @@
+/*
+ * bq.h - blockwise codebook quantization / dequantization and GGUF
+ * Q8_0 / Q4_0 dequantization on NVIDIA B200 (sm_100a).  C ABI of libbq.so.
+ *
+ * Common contract of every compute entry point
+ * -------------------------------------------
+ *  - All data pointers are DEVICE pointers on the current CUDA device, owned
+ *    and allocated by the caller.  The library allocates nothing, copies
+ *    nothing from the host, and never synchronizes.
+ *  - All work is enqueued on `stream`, which may be the legacy default stream
+ *    (0) if the caller passes it; nothing is ever launched on any other
+ *    stream.  This is the stream contract of "bitsandbytes PR #2052, Respect
+ *    the current CUDA stream in blockwise quantization" (Summary: launches on
+ *    the legacy default stream raced producers on PyTorch's current stream).
+ *    Inputs must stay valid and unmodified until the stream work completes.
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns BQ_ERR_INVALID_ARG (or BQ_ERR_UNSUPPORTED) and leaves
+ *    every buffer untouched.  n == 0 (or n_blocks == 0) returns BQ_OK with no
+ *    launch.  A failed launch returns BQ_ERR_CUDA; bq_last_cuda_error() then
+ *    gives the CUDA message (per calling thread).  Faults during execution
+ *    surface at the caller's next synchronization, as with any CUDA work.
+ *  - Any pointer alignment allowed by the element type is accepted.  16-byte
+ *    aligned buffers take the vectorised / TMA path; others a scalar path with
+ *    identical results.
+ *  - Thread safety: entry points may be called concurrently from several host
+ *    threads (no shared host state besides the per-thread error text).
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define BQ_API __attribute__((visibility("default")))
+#else
+#define BQ_API
+#endif
+
+typedef enum bq_status {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1,   /* bad size, pointer, blocksize or codebook length */
+    BQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement     */
+    BQ_ERR_CUDA = 3           /* a CUDA call failed; see bq_last_cuda_error()    */
+} bq_status;
+
+/* Element types of inputs (quantize) and outputs (dequantize). */
+typedef enum bq_dtype {
+    BQ_F32 = 0,               /* IEEE binary32                    */
+    BQ_F16 = 1,               /* IEEE binary16                    */
+    BQ_BF16 = 2               /* bfloat16 (top half of a binary32) */
+} bq_dtype;
+
+/*
+ * Blockwise absmax codebook quantization.
+ * Defined by "bitsandbytes PR #2052" (Summary: General8, FP4 and NF4 blockwise
+ * quantization; Correctness: FP16/BF16/FP32 inputs, every block size from 32
+ * through 4096, full blocks and tails).
+ *
+ * For block b = elements [b*blocksize, min(n, (b+1)*blocksize)):
+ *   absmax[b] = max |x_i|                          (fp32; +0 for an all-zero block)
+ *   xn_i      = absmax[b] == 0 ? 0 : x_i / absmax[b]   (fp32, IEEE division)
+ *   idx_i     = argmin_j |RN(xn_i - code[j])|      (fp32; lowest j on ties)
+ *
+ *   x            device, n elements of x_dtype, contiguous.
+ *   n            element count, >= 0.
+ *   blocksize    power of two in [32, 4096].
+ *   code         device, code_entries fp32 values sorted ascending (non-decreasing);
+ *                finite.  16 entries -> 4-bit codes, 256 entries -> 8-bit codes.
+ *                Unsorted tables are accepted and still give the exact result,
+ *                on a slow path (sortedness is checked on the device).
+ *   absmax       device, ceil(n / blocksize) fp32, written.
+ *   out          device, written: 16 entries: ceil(n/2) bytes, element 2i in the
+ *                high nibble of byte i, element 2i+1 in the low nibble (0 if it
+ *                does not exist); 256 entries: n bytes, one code per element.
+ * Inputs must be finite (non-finite values are outside the contract).
+ */
+BQ_API bq_status bq_quantize_blockwise(const void *x, bq_dtype x_dtype, int64_t n,
+                                int32_t blocksize, const float *code,
+                                int32_t code_entries, float *absmax,
+                                uint8_t *out, cudaStream_t stream);
+
+/*
+ * Blockwise dequantization, the inverse map of bq_quantize_blockwise:
+ *   y_i = narrow_to(y_dtype, RN(code[idx_i] * absmax[i / blocksize]))
+ * with one fp32 product and one round-to-nearest-even narrowing.
+ *   q        device, packed codes laid out as `out` above.
+ *   absmax   device, ceil(n / blocksize) fp32.
+ *   code     device, code_entries (16 or 256) fp32 values (any order).
+ *   y        device, n elements of y_dtype, written.
+ */
+BQ_API bq_status bq_dequantize_blockwise(const uint8_t *q, const float *absmax,
+                                  int64_t n, int32_t blocksize,
+                                  const float *code, int32_t code_entries,
+                                  void *y, bq_dtype y_dtype,
+                                  cudaStream_t stream);
+
+/*
+ * GGUF Q8_0 dequantization ("ComfyUI-GGUF PR #472, Cache device-side
+ * constants in dequant kernels", Verification table, Q8_0 row: the one type
+ * with no shift constant).  Block k is 34 bytes: fp16 d (little endian, bytes
+ * 0..1) then 32 signed bytes q_j.  y[32k + j] = narrow_to(y_dtype, d * q_j);
+ * the fp32 product is exact.
+ *   blocks   device, n_blocks * 34 bytes (any byte alignment).
+ *   y        device, 32 * n_blocks elements of y_dtype, written.
+ */
+BQ_API bq_status bq_dequant_q8_0(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * GGUF Q4_0 dequantization (same page, Problem section: each quant byte is
+ * split by the shift vector [0, 4], low nibbles first).  Block k is 18 bytes:
+ * fp16 d then 16 bytes qs.  For j < 16:
+ *   y[32k + j]      = narrow_to(y_dtype, d * ((qs[j] & 15) - 8))
+ *   y[32k + 16 + j] = narrow_to(y_dtype, d * ((qs[j] >> 4) - 8))
+ *   blocks   device, n_blocks * 18 bytes (any byte alignment).
+ *   y        device, 32 * n_blocks elements of y_dtype, written.
+ */
+BQ_API bq_status bq_dequant_q4_0(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/* Static text for a status code. */
+BQ_API const char *bq_status_string(bq_status s);
+
+/* Text of the last CUDA error seen by an entry point on this host thread
+ * ("" if none).  The pointer stays valid until the next call on this thread. */
+BQ_API const char *bq_last_cuda_error(void);
+
+/*
+ * Device-side fault word.  Kernels that wait on an mbarrier give up after a
+ * bounded time instead of hanging, set a bit here and return; results of that
+ * launch are then invalid.  Reads the word of the current device (this call
+ * SYNCHRONIZES the device), stores it in *fault and, if reset != 0, clears it.
+ * 0 means no fault was recorded.
+ */
+BQ_API bq_status bq_device_fault(uint32_t *fault, int32_t reset);
+
+/* BQ_ABI_VERSION of the loaded library. */
+BQ_API int32_t bq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BQ_H */

@@ -1,0 +1,239 @@
+// bq_probes.cu - test-only CUDA checks of the library's exact arithmetic.
+//
+// 1. Division: the normalisation the quantize kernels use (per-block
+//    reciprocal + Markstein correction, IEEE division for the small-|x| and
+//    out-of-range cases) against IEEE division, for every pair of finite
+//    bf16 / fp16 values (x, A) with 0 < A and |x| <= A, and for random and
+//    edge-heavy fp32 pairs.
+// 2. Search: the fast nearest-code search (bucket table or threshold
+//    bisection, built on the device from the caller's table) against a plain
+//    linear scan of the rule |RN(xn - c_j)| minimal, lowest j on ties, for
+//    EVERY float xn in [-1, 1].
+//
+// The plain scan here is written independently of the library's code.
+#include <cstdint>
+
+#include "bq_search.cuh"
+
+namespace {
+
+__device__ unsigned long long g_mismatch;
+__device__ unsigned int g_first_bad_a;
+__device__ unsigned int g_first_bad_b;
+
+__device__ __forceinline__ bool same_quotient(float a, float b) {
+  // the sign of a zero quotient does not matter to the search
+  return __float_as_uint(a) == __float_as_uint(b) || (a == 0.0f && b == 0.0f);
+}
+
+__device__ __forceinline__ float kernel_division(float x, float A) {
+  const bq::BlockScale s = bq::make_scale(A);
+  return fabsf(x) < s.theta ? bq::div_exact(x, A) : bq::div_fast(x, s);
+}
+
+__device__ void report(unsigned int a, unsigned int b) {
+  if (atomicAdd(&g_mismatch, 1ull) == 0ull) {
+    g_first_bad_a = a;
+    g_first_bad_b = b;
+  }
+}
+
+// 16-bit types: thread handles A = pattern blockIdx-derived, x over all.
+template <int DT>
+__global__ void div16_all(int a_lo) {
+  const uint32_t a_bits = static_cast<uint32_t>(a_lo) + blockIdx.x;
+  const float A = bq::widen_pair_elem<DT>(a_bits, 0);
+  if (!(A > 0.0f) || !isfinite(A)) return;
+  for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+    const float x = bq::widen_pair_elem<DT>(xb, 0);
+    if (!isfinite(x) || !(fabsf(x) <= A)) continue;
+    const float got = kernel_division(x, A);
+    const float want = __fdiv_rn(x, A);
+    if (!same_quotient(got, want)) report(xb, a_bits);
+  }
+}
+
+__device__ __forceinline__ uint32_t mix(uint64_t v) {
+  v ^= v >> 33; v *= 0xff51afd7ed558ccdull;
+  v ^= v >> 33; v *= 0xc4ceb9fe1a85ec53ull;
+  v ^= v >> 33;
+  return static_cast<uint32_t>(v);
+}
+
+__global__ void div32_random(uint64_t count, uint64_t seed) {
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += stride) {
+    uint32_t ab = mix(seed + 2 * i), xb = mix(seed + 2 * i + 1);
+    const uint32_t kind = i & 3;
+    if (kind == 1) ab |= 0x007fffffu;            // all-ones mantissa
+    if (kind == 2) xb |= 0x007fffffu;
+    if (kind == 3) ab = (ab & 0xff800000u) | 0x00000001u;
+    ab &= 0x7fffffffu;
+    float A = __uint_as_float(ab);
+    float x = __uint_as_float(xb);
+    if (!isfinite(A) || !isfinite(x) || A == 0.0f) continue;
+    if (fabsf(x) > A) { const float t = A; A = fabsf(x); x = copysignf(t, x); }
+    const float got = kernel_division(x, A);
+    const float want = __fdiv_rn(x, A);
+    if (!same_quotient(got, want)) report(__float_as_uint(x), __float_as_uint(A));
+  }
+}
+
+// ------------------------------------------------------------- search ----
+
+template <int E>
+struct ProbeSmem {
+  bq::TableSmem tab;
+  bq::Lut<E> lut;
+  float c[E];
+};
+
+template <int E>
+__device__ uint32_t plain_scan(float xn, const float* c) {
+  uint32_t best_j = 0;
+  float best = fabsf(__fsub_rn(xn, c[0]));
+  for (int j = 1; j < E; ++j) {
+    const float d = fabsf(__fsub_rn(xn, c[j]));
+    if (d < best) { best = d; best_j = j; }
+  }
+  return best_j;
+}
+
+// Every float in [-1, 1]: positive bit patterns 0..0x3f800000 and their negatives.
+template <int E>
+__global__ void __launch_bounds__(256) search_all(const float* code, int* mode_out) {
+  extern __shared__ uint8_t raw[];
+  ProbeSmem<E>& s = *reinterpret_cast<ProbeSmem<E>*>(raw);
+  const int ct = threadIdx.x;
+  bq::build_search<E>(s.tab, s.lut, code, ct);
+  if (ct < E) s.c[ct] = code[ct];
+  __syncthreads();
+  const int mode = s.tab.mode;
+  if (blockIdx.x == 0 && ct == 0) *mode_out = mode;
+  const uint64_t npos = 0x3f800001ull;
+  const uint64_t total = 2 * npos;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + ct; i < total; i += stride) {
+    const uint32_t bits = i < npos ? static_cast<uint32_t>(i)
+                                   : (static_cast<uint32_t>(i - npos) | 0x80000000u);
+    const float xn = __uint_as_float(bits);
+    uint32_t got;
+    if (mode == bq::kModeLut) got = bq::search<E, bq::kModeLut>(xn, s.tab, s.lut);
+    else if (mode == bq::kModeBsearch) got = bq::search<E, bq::kModeBsearch>(xn, s.tab, s.lut);
+    else got = bq::search<E, bq::kModeScan>(xn, s.tab, s.lut);
+    const uint32_t want = plain_scan<E>(xn, s.c);
+    if (got != want) report(bits, (got << 16) | want);
+  }
+}
+
+template <int E, int MODE>
+__global__ void __launch_bounds__(256) search_forced(const float* code, int* mode_out) {
+  // same sweep, but with a forced search form (to test the bisection form too)
+  extern __shared__ uint8_t raw[];
+  ProbeSmem<E>& s = *reinterpret_cast<ProbeSmem<E>*>(raw);
+  const int ct = threadIdx.x;
+  bq::build_search<E>(s.tab, s.lut, code, ct);
+  if (ct < E) s.c[ct] = code[ct];
+  __syncthreads();
+  if (blockIdx.x == 0 && ct == 0) *mode_out = s.tab.mode;
+  if (s.tab.mode == bq::kModeScan) return;   // forced forms need a valid table
+  const uint64_t npos = 0x3f800001ull;
+  const uint64_t total = 2 * npos;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + ct; i < total; i += stride) {
+    const uint32_t bits = i < npos ? static_cast<uint32_t>(i)
+                                   : (static_cast<uint32_t>(i - npos) | 0x80000000u);
+    const float xn = __uint_as_float(bits);
+    const uint32_t got = bq::search<E, MODE>(xn, s.tab, s.lut);
+    const uint32_t want = plain_scan<E>(xn, s.c);
+    if (got != want) report(bits, (got << 16) | want);
+  }
+}
+
+int g_sms = 0;
+
+cudaError_t reset() {
+  unsigned long long z = 0;
+  unsigned int zi = 0;
+  cudaError_t e = cudaMemcpyToSymbol(g_mismatch, &z, sizeof(z));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_first_bad_a, &zi, sizeof(zi));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_first_bad_b, &zi, sizeof(zi));
+  if (e == cudaSuccess && g_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  return e;
+}
+
+int finish(unsigned long long* mismatches, unsigned int* first_a, unsigned int* first_b) {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(mismatches, g_mismatch, sizeof(*mismatches));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(first_a, g_first_bad_a, sizeof(*first_a));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(first_b, g_first_bad_b, sizeof(*first_b));
+  return static_cast<int>(e);
+}
+
+// mode_out is a HOST pointer: the kernel writes the chosen search form into a
+// device word, copied back after the sweep.
+template <int E, typename K>
+int run_search(K kernel, const float* code, int* mode_out, unsigned long long* mm,
+               unsigned int* fa, unsigned int* fb) {
+  cudaError_t e = reset();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const size_t smem = sizeof(ProbeSmem<E>);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  int* d_mode = nullptr;
+  e = cudaMalloc(&d_mode, sizeof(int));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  kernel<<<g_sms * 4, 256, smem>>>(code, d_mode);
+  int rc = finish(mm, fa, fb);
+  if (rc == 0) rc = static_cast<int>(cudaMemcpy(mode_out, d_mode, sizeof(int), cudaMemcpyDeviceToHost));
+  cudaFree(d_mode);
+  return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+// dtype: 1 = fp16, 2 = bf16.  Returns a cudaError_t value.
+__attribute__((visibility("default"))) int probe_div16(int dtype, unsigned long long* mm,
+                                                       unsigned int* fa, unsigned int* fb) {
+  cudaError_t e = reset();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  // A over all positive patterns 0x0001..0x7fff (65535 CTAs)
+  if (dtype == 1) div16_all<bq::kF16><<<0x7fff, 256>>>(1);
+  else div16_all<bq::kBF16><<<0x7fff, 256>>>(1);
+  return finish(mm, fa, fb);
+}
+
+__attribute__((visibility("default"))) int probe_div32(unsigned long long count,
+                                                       unsigned long long seed,
+                                                       unsigned long long* mm, unsigned int* fa,
+                                                       unsigned int* fb) {
+  cudaError_t e = reset();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  div32_random<<<g_sms * 8, 256>>>(count, seed);
+  return finish(mm, fa, fb);
+}
+
+// mode_request: -1 = whatever the builder picks, 1 = force the bisection form.
+__attribute__((visibility("default"))) int probe_search(const float* code, int entries,
+                                                        int mode_request, int* mode_out,
+                                                        unsigned long long* mm, unsigned int* fa,
+                                                        unsigned int* fb) {
+  if (entries == 16) {
+    if (mode_request == 1)
+      return run_search<16>(search_forced<16, bq::kModeBsearch>, code, mode_out, mm, fa, fb);
+    return run_search<16>(search_all<16>, code, mode_out, mm, fa, fb);
+  }
+  if (mode_request == 1)
+    return run_search<256>(search_forced<256, bq::kModeBsearch>, code, mode_out, mm, fa, fb);
+  return run_search<256>(search_all<256>, code, mode_out, mm, fa, fb);
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+"""The C-ABI library: it loads, exports every symbol include/bq.h declares,
+and validates arguments on the host before any CUDA call (so these run
+without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dequantization_bq_quantize_b200 as bq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "bq.h")).read()
+    return re.findall(r"BQ_API\s+[\w\s\*]+?\b(bq_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def L():
+    bq.build()
+    return bq.lib()
+
+
+def test_header_declares_the_four_calls():
+    syms = declared_symbols()
+    for name in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
+                 "bq_dequant_q4_0"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(L):
+    syms = declared_symbols()
+    assert len(syms) >= 8
+    for name in syms:
+        assert hasattr(L, name), name
+        assert name in bq.EXPORTED
+
+
+def test_abi_version_and_status_strings(L):
+    assert bq.bq_abi_version() == 1
+    assert bq.bq_status_string(bq.BQ_OK) == "ok"
+    assert bq.bq_status_string(bq.BQ_ERR_INVALID_ARG) == "invalid argument"
+    assert bq.bq_status_string(bq.BQ_ERR_CUDA) == "CUDA error"
+    assert bq.bq_status_string(99) == "unknown status"
+
+
+P = 0x10000  # a fake, 64 KiB-aligned device address: never dereferenced here
+
+
+@pytest.mark.parametrize("bs", [0, 16, 48, 8192, -64, 100])
+def test_rejects_bad_blocksize(L, bs):
+    assert bq.bq_quantize_blockwise(P, bq.BQ_BF16, 100, bs, P, 16, P, P, 0) == bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_dequantize_blockwise(P, P, 100, bs, P, 16, P, bq.BQ_BF16, 0) == bq.BQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("entries", [0, 8, 15, 17, 255, 512])
+def test_rejects_bad_codebook_length(L, entries):
+    assert bq.bq_quantize_blockwise(P, bq.BQ_F32, 100, 64, P, entries, P, P, 0) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_rejects_bad_sizes_pointers_dtypes(L):
+    E = bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_quantize_blockwise(P, bq.BQ_F32, -1, 64, P, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(P, 7, 100, 64, P, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(0, bq.BQ_F32, 100, 64, P, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(P, bq.BQ_F32, 100, 64, 0, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(P, bq.BQ_F32, 100, 64, P, 16, 0, P, 0) == E
+    assert bq.bq_quantize_blockwise(P, bq.BQ_F32, 100, 64, P, 16, P, 0, 0) == E
+    # element misaligned for its type
+    assert bq.bq_quantize_blockwise(P + 2, bq.BQ_F32, 100, 64, P, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(P + 1, bq.BQ_BF16, 100, 64, P, 16, P, P, 0) == E
+    assert bq.bq_quantize_blockwise(P, bq.BQ_BF16, 100, 64, P, 16, P + 2, P, 0) == E
+    assert bq.bq_dequantize_blockwise(P, P, 100, 64, P, 16, P + 1, bq.BQ_F16, 0) == E
+    assert bq.bq_dequantize_blockwise(0, P, 100, 64, P, 16, P, bq.BQ_F16, 0) == E
+    assert bq.bq_dequant_q8_0(P, -1, P, bq.BQ_BF16, 0) == E
+    assert bq.bq_dequant_q4_0(0, 10, P, bq.BQ_BF16, 0) == E
+    assert bq.bq_dequant_q4_0(P, 10, P + 1, bq.BQ_BF16, 0) == E
+    assert bq.bq_dequant_q4_0(P, 10, P, 9, 0) == E
+
+
+def test_zero_length_is_ok_without_touching_the_device(L):
+    # n == 0 returns before any CUDA call, even with null buffers
+    assert bq.bq_quantize_blockwise(0, bq.BQ_F32, 0, 64, 0, 16, 0, 0, 0) == bq.BQ_OK
+    assert bq.bq_dequantize_blockwise(0, 0, 0, 64, 0, 256, 0, bq.BQ_BF16, 0) == bq.BQ_OK
+    assert bq.bq_dequant_q8_0(0, 0, 0, bq.BQ_BF16, 0) == bq.BQ_OK
+    assert bq.bq_dequant_q4_0(0, 0, 0, bq.BQ_F32, 0) == bq.BQ_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(bq, "_lib", None)
+    monkeypatch.setattr(bq, "LIB_PATH", str(tmp_path / "libbq.so"))
+    with pytest.raises(ImportError):
+        bq.lib()
+
+
+def test_library_has_no_oracle_dependency(L):
+    # the product library links neither the oracle nor anything under tests/
+    out = os.popen(f"ldd {bq.LIB_PATH} 2>/dev/null").read()
+    assert "oracle" not in out
+    src = open(os.path.join(ROOT, "dequantization_bq_quantize_b200", "__init__.py")).read()
+    assert "import oracle" not in src and "from oracle" not in src

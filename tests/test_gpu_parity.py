@@ -1,0 +1,374 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Codes, packed bytes and absmax must match bit for bit; dequantized values
+must match exactly (the contract allows 1 ulp for bf16/fp16; the kernels do the
+same single product and rounding, so exact equality is asserted).
+"""
+import ctypes
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import dequantization_bq_quantize_b200 as bq
+import oracle
+from bq_inputs import codebooks, synth
+
+from gpu_util import Guarded, device_copy, np_bits, sample_blocks
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DT_CODE = {"f32": bq.BQ_F32, "f16": bq.BQ_F16, "bf16": bq.BQ_BF16}
+EB = {"f32": 4, "f16": 2, "bf16": 2}
+TABLES = {name: codebooks.get(name) for name in ("nf4", "fp4", "dyn8")}
+BLOCKSIZES = [32, 64, 128, 256, 512, 1024, 2048, 4096]
+
+
+@pytest.fixture(autouse=True)
+def _no_fault():
+    bq.bq_device_fault(reset=True)
+    yield
+    assert bq.bq_device_fault(reset=True) == 0, "a kernel gave up waiting (fault word set)"
+
+
+def code_dev(table):
+    return torch.from_numpy(np.ascontiguousarray(table, np.float32)).cuda()
+
+
+def gpu_quantize(x_np, dtype, bs, table, x_offset=0, out_offset=0, stream=0):
+    """Quantize host array x_np (oracle conventions) on the GPU through the
+    C ABI; returns (absmax, codes) as numpy plus guard status."""
+    n = x_np.size
+    xt, xp = device_copy(x_np, x_offset)
+    code = code_dev(table)
+    nb = (n + bs - 1) // bs
+    amax = Guarded(4 * nb)
+    out = Guarded(oracle.code_bytes(n, table.size), out_offset)
+    st = bq.bq_quantize_blockwise(xp, DT_CODE[dtype], n, bs, code.data_ptr(), table.size,
+                                  amax.ptr, out.ptr, stream)
+    assert st == bq.BQ_OK, (st, bq.bq_last_cuda_error())
+    torch.cuda.synchronize()
+    assert amax.guards_intact() and out.guards_intact()
+    return amax.host().view(np.float32), out.host(), (xt, code)
+
+
+def gpu_dequantize(q_np, amax_np, n, bs, table, ydtype, y_offset=0, q_offset=0):
+    qt, qp = device_copy(q_np, q_offset)
+    at, ap = device_copy(amax_np)
+    code = code_dev(table)
+    y = Guarded(EB[ydtype] * n, y_offset)
+    st = bq.bq_dequantize_blockwise(qp, ap, n, bs, code.data_ptr(), table.size, y.ptr,
+                                    DT_CODE[ydtype], 0)
+    assert st == bq.BQ_OK, (st, bq.bq_last_cuda_error())
+    torch.cuda.synchronize()
+    assert y.guards_intact()
+    h = y.host()
+    return h.view(np.float32) if ydtype == "f32" else h.view(np.uint16)
+
+
+def check_quant(x_np, dtype, bs, name, **kw):
+    table = TABLES[name]
+    ga, go, _ = gpu_quantize(x_np, dtype, bs, table, **kw)
+    oa, oo = oracle.quantize_blockwise(x_np, dtype, bs, table)
+    assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32)), "absmax differs"
+    bad = np.nonzero(go != oo)[0]
+    assert bad.size == 0, f"{bad.size} code bytes differ, first at {bad[:5]}: gpu {go[bad[:5]]} oracle {oo[bad[:5]]}"
+    return oa, oo
+
+
+def check_dequant(q, amax, n, bs, name, ydtype, **kw):
+    table = TABLES[name]
+    gy = gpu_dequantize(q, amax, n, bs, table, ydtype, **kw)
+    oy = oracle.dequantize_blockwise(q, amax, n, bs, table, ydtype)
+    bad = np.nonzero(gy.view(np.uint32 if ydtype == "f32" else np.uint16) !=
+                     oy.view(np.uint32 if ydtype == "f32" else np.uint16))[0]
+    assert bad.size == 0, f"{bad.size} dequantized values differ, first at {bad[:5]}"
+
+
+def small_input(n, dtype, bs, seed):
+    """N(0,1) with one all-zero block, a block of outliers, exact table values."""
+    x = synth.normal(n, dtype, seed).float()
+    nb = (n + bs - 1) // bs
+    if nb > 2:
+        x[(nb // 2) * bs: min(n, (nb // 2 + 1) * bs)] = 0
+        x[bs: 2 * bs] *= 50.0
+    return np_bits(x.to(synth.TORCH_DTYPES[dtype]))
+
+
+# ------------------------------------------------------------ small sweep --
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("name", ["nf4", "fp4", "dyn8"])
+@pytest.mark.parametrize("bs", BLOCKSIZES)
+def test_quantize_dequantize_parity_small(dtype, name, bs):
+    # several 16 KiB tiles plus a ragged tail of whole and partial blocks
+    n = 5 * 8192 + 3 * bs + 37 if dtype != "f32" else 9 * 4096 + 3 * bs + 37
+    x = small_input(n, dtype, bs, seed=bs + 7 * len(name))
+    oa, oo = check_quant(x, dtype, bs, name)
+    for ydtype in ("f32", "bf16", "f16"):
+        check_dequant(oo, oa, n, bs, name, ydtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("name", ["nf4", "dyn8"])
+def test_edge_sizes(dtype, name):
+    for bs in (32, 64, 4096):
+        for n in (1, 2, 3, 31, 32, 33, bs - 1, bs, bs + 1, 2 * bs + 37):
+            x = small_input(n, dtype, bs, seed=n)
+            oa, oo = check_quant(x, dtype, bs, name)
+            check_dequant(oo, oa, n, bs, name, dtype)
+
+
+@pytest.mark.parametrize("name", ["nf4", "dyn8"])
+def test_unaligned_pointers(name):
+    n, bs = 3 * 8192 + 101, 64
+    x = small_input(n, "bf16", bs, seed=3)
+    for x_off, o_off in ((2, 0), (0, 1), (6, 3), (16, 8)):
+        check_quant(x, "bf16", bs, name, x_offset=x_off, out_offset=o_off)
+    oa, oo = oracle.quantize_blockwise(x, "bf16", bs, TABLES[name])
+    for y_off, q_off in ((2, 0), (0, 1), (8, 2)):
+        check_dequant(oo, oa, n, bs, name, "bf16", y_offset=y_off, q_offset=q_off)
+
+
+def test_special_values_and_ties():
+    """Exact codebook values, midpoints between entries and their neighbours,
+    tiny and huge magnitudes (the IEEE-division fallback), fp32."""
+    rng = np.random.default_rng(11)
+    for name in ("nf4", "fp4", "dyn8"):
+        t = TABLES[name].astype(np.float64)
+        mids = ((t[:-1] + t[1:]) / 2).astype(np.float32)
+        vals = np.concatenate([t.astype(np.float32), mids, np.nextafter(mids, np.float32(2)),
+                               np.nextafter(mids, np.float32(-2))])
+        bs = 64
+        blocks = []
+        for scale in (1.0, 3.0, 1e-30, 1e30, 2.0 ** -126, 7.25):
+            v = (vals * np.float32(scale)).astype(np.float32)
+            for k in range(0, v.size, bs - 1):
+                blk = np.zeros(bs, np.float32)
+                part = v[k:k + bs - 1]
+                blk[:part.size] = part
+                blk[bs - 1] = np.float32(scale)            # absmax = scale
+                blocks.append(blk)
+        # blocks with a huge dynamic range: |x| far below absmax * 2^-40
+        for _ in range(8):
+            blk = (rng.standard_normal(bs) * np.exp(rng.uniform(-80, 0, bs))).astype(np.float32)
+            blk[0] = 1.0
+            blocks.append(blk)
+        x = np.concatenate(blocks)
+        oa, oo = check_quant(x, "f32", bs, name)
+        check_dequant(oo, oa, x.size, bs, name, "f32")
+
+
+def test_unsorted_and_tight_tables():
+    """Tables the fast search does not accept: unsorted (plain scan) and
+    tightly spaced (bisection or scan) still give the rule's result."""
+    n, bs = 2 * 8192 + 77, 64
+    x = small_input(n, "bf16", bs, seed=21)
+    rng = np.random.default_rng(2)
+    perm = TABLES["nf4"][rng.permutation(16)]
+    tight = np.sort(np.concatenate([np.linspace(-1, 1, 15), [1e-7]])).astype(np.float32)
+    dup = np.sort(np.concatenate([TABLES["nf4"][:12], [0.5, 0.5, 0.5, 1.0]])).astype(np.float32)
+    lin256 = np.linspace(-1, 1, 256).astype(np.float32)
+    for table in (perm, tight, dup, lin256):
+        ga, go, _ = gpu_quantize(x, "bf16", bs, table)
+        oa, oo = oracle.quantize_blockwise(x, "bf16", bs, table)
+        assert np.array_equal(ga, oa) and np.array_equal(go, oo)
+
+
+def test_zero_length_and_bad_arguments():
+    code = code_dev(TABLES["nf4"])
+    amax = torch.empty(4, device="cuda")
+    out = torch.empty(64, dtype=torch.uint8, device="cuda")
+    x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    assert bq.bq_quantize_blockwise(x.data_ptr(), bq.BQ_BF16, 0, 64, code.data_ptr(), 16,
+                                    amax.data_ptr(), out.data_ptr(), 0) == bq.BQ_OK
+    assert bq.bq_quantize_blockwise(x.data_ptr(), bq.BQ_BF16, 64, 48, code.data_ptr(), 16,
+                                    amax.data_ptr(), out.data_ptr(), 0) == bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_quantize_blockwise(x.data_ptr() + 1, bq.BQ_BF16, 64, 64, code.data_ptr(), 16,
+                                    amax.data_ptr(), out.data_ptr(), 0) == bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_dequant_q8_0(0, 5, out.data_ptr(), bq.BQ_BF16, 0) == bq.BQ_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------- stream order --
+
+def _ordering_case(use_callers_stream):
+    """A producer fills the input on a non-blocking stream held back by a
+    ~25 ms device-side delay, then quantize is called at once."""
+    n, bs = 1 << 20, 64
+    code = code_dev(TABLES["nf4"])
+    x_final = small_input(n, "bf16", bs, seed=5)
+    src = torch.from_numpy(x_final.view(np.int16)).cuda()
+    x = torch.zeros(n, dtype=torch.int16, device="cuda")
+    amax = torch.empty((n + bs - 1) // bs, device="cuda")
+    out = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()  # non-blocking with respect to the legacy stream
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(50_000_000)  # bounded spin, tens of ms
+        x.copy_(src)
+        st = bq.bq_quantize_blockwise(x.data_ptr(), bq.BQ_BF16, n, bs, code.data_ptr(), 16,
+                                      amax.data_ptr(), out.data_ptr(),
+                                      s.cuda_stream if use_callers_stream else 0)
+    assert st == bq.BQ_OK
+    torch.cuda.synchronize()
+    oa, oo = oracle.quantize_blockwise(x_final, "bf16", bs, TABLES["nf4"])
+    return np.array_equal(amax.cpu().numpy(), oa) and np.array_equal(out.cpu().numpy(), oo)
+
+
+def test_respects_callers_stream():
+    """Ordering regression of the stream-aware entry points (bitsandbytes
+    PR #2052): on the caller's stream the quantizer sees the final input."""
+    assert _ordering_case(True)
+
+
+def test_ordering_case_detects_wrong_stream():
+    """Control: the same sequence with the legacy stream reads stale input,
+    so the case above can tell the two apart."""
+    assert not _ordering_case(False)
+
+
+# ------------------------------------------------------------------ GGUF --
+
+@pytest.mark.parametrize("kind", ["q8_0", "q4_0"])
+@pytest.mark.parametrize("ydtype", ["bf16", "f16", "f32"])
+def test_gguf_parity(kind, ydtype):
+    bb = 34 if kind == "q8_0" else 18
+    fn = bq.bq_dequant_q8_0 if kind == "q8_0" else bq.bq_dequant_q4_0
+    ofn = oracle.dequant_q8_0 if kind == "q8_0" else oracle.dequant_q4_0
+    for nblk, off in ((4096, 0), (4096 * 14336 // 32, 0), (1, 0), (7, 0), (8, 0), (9, 0),
+                      (1000 + 3, 0), (1003, 2), (517, 1), (64, 16)):
+        blocks = synth.gguf_blocks(nblk, kind, seed=4 + nblk)
+        bt, bp = device_copy(blocks, off)
+        y = Guarded(EB[ydtype] * 32 * nblk)
+        assert fn(bp, nblk, y.ptr, DT_CODE[ydtype], 0) == bq.BQ_OK
+        torch.cuda.synchronize()
+        assert y.guards_intact()
+        got = y.host().view(np.float32 if ydtype == "f32" else np.uint16)
+        want = ofn(blocks, ydtype)
+        assert np.array_equal(got, want), (kind, nblk, off)
+
+
+def test_gguf_hand_blocks_on_gpu():
+    import test_oracle_pins as pins
+    for kind, blk, expect in pins._load_hand_blocks():
+        fn = bq.bq_dequant_q8_0 if kind == "q8_0" else bq.bq_dequant_q4_0
+        bt, bp = device_copy(blk)
+        y = Guarded(4 * 32)
+        assert fn(bp, 1, y.ptr, bq.BQ_F32, 0) == bq.BQ_OK
+        torch.cuda.synchronize()
+        assert np.array_equal(y.host().view(np.uint32), expect.view(np.uint32))
+
+
+# ------------------------------------------------------ full-size configs --
+
+def _run_full(x_cpu, dtype, bs, name, sample=3000, seed=0):
+    """Full-size run through the torch helpers (same launch configuration as
+    the benchmark), checked on sampled whole blocks against the oracle and on
+    all blocks for properties that hold at any size."""
+    table = TABLES[name]
+    code = code_dev(table)
+    n = x_cpu.numel()
+    x = x_cpu.cuda()
+    amax, q = bq.quantize_blockwise(x, code, bs)
+    y = bq.dequantize_blockwise(q, amax, n, bs, code, dtype=x.dtype)
+    torch.cuda.synchronize()
+    nb = amax.numel()
+    # properties at any size: absmax is max|x| of each block, dequant of the
+    # block's extreme element is +-absmax * (table end) ...
+    xf = x.float()
+    full_blocks = n // bs
+    ref_amax = xf[: full_blocks * bs].abs().view(full_blocks, bs).amax(dim=1)
+    assert torch.equal(amax[:full_blocks], ref_amax)
+    # sampled blocks against the oracle
+    xh = np_bits(x_cpu)
+    ah, qh, yh = amax.cpu().numpy(), q.cpu().numpy(), np_bits(y.cpu())
+    for b in sample_blocks(nb, sample, seed):
+        lo, hi = b * bs, min(n, (b + 1) * bs)
+        oa, oo = oracle.quantize_blockwise(xh[lo:hi], dtype, bs, table)
+        assert ah[b] == oa[0]
+        q0 = lo // 2 if table.size == 16 else lo
+        assert np.array_equal(qh[q0:q0 + oo.size], oo), b
+        oy = oracle.dequantize_blockwise(oo, oa, hi - lo, bs, table, dtype)
+        assert np.array_equal(yh[lo:hi], oy), b
+
+
+def test_config_small_fp32_nf4_full():
+    """n = 65536 fp32 N(0,1), NF4, blocksize 64: every byte against the oracle."""
+    x = np_bits(synth.normal(synth.SMALL_N, "f32", 0))
+    oa, oo = check_quant(x, "f32", 64, "nf4")
+    check_dequant(oo, oa, x.size, 64, "nf4", "f32")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("name", ["nf4", "fp4", "dyn8"])
+def test_config_sweep_sampled(dtype, name):
+    """The 45-cell sweep at n = 8388608 + 37 with one all-zero block."""
+    for i, bs in enumerate((32, 64, 256, 1024, 4096)):
+        cell = ["f16", "bf16", "f32"].index(dtype) * 15 + ["nf4", "fp4", "dyn8"].index(name) * 5 + i
+        x = synth.sweep(dtype, bs, seed=1 + cell)
+        _run_full(x, dtype, bs, name, sample=400, seed=cell)
+
+
+def test_config_large_bf16_nf4():
+    """bf16 n = 2^29 (1 GiB) N(0, 0.02) with 0.1% outliers, NF4, blocksize 64."""
+    x, count = synth.large_outliers()
+    assert 0.0009 < count / x.numel() < 0.0011
+    _run_full(x, "bf16", 64, "nf4", sample=4000, seed=3)
+
+
+def test_config_llama_weight_set_sampled():
+    """A few of the Llama-3-8B-shaped matrices (bf16 N(0, 0.02), NF4 bs 64)."""
+    mats = synth.llama_matrices(layers=32)
+    for layer, i, name, r, c, seed in (mats[0], mats[4], mats[6], mats[-1]):
+        x = synth.normal(r * c, "bf16", seed, std=0.02)
+        _run_full(x, "bf16", 64, "nf4", sample=300, seed=seed)
+
+
+# ---------------------------------------------------------- exhaustive ----
+
+@pytest.fixture(scope="module")
+def probes():
+    import os
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), "gpu_probes"))
+    import build as pbuild
+    L = ctypes.CDLL(pbuild.build())
+    u64p, u32p = ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_uint)
+    L.probe_div16.argtypes = [ctypes.c_int, u64p, u32p, u32p]
+    L.probe_div32.argtypes = [ctypes.c_ulonglong, ctypes.c_ulonglong, u64p, u32p, u32p]
+    L.probe_search.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                               ctypes.POINTER(ctypes.c_int), u64p, u32p, u32p]
+    return L
+
+
+def _outs():
+    return ctypes.c_ulonglong(0), ctypes.c_uint(0), ctypes.c_uint(0)
+
+
+@pytest.mark.parametrize("dt", [1, 2], ids=["f16", "bf16"])
+def test_division_exhaustive_16bit(probes, dt):
+    mm, fa, fb = _outs()
+    assert probes.probe_div16(dt, ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
+    assert mm.value == 0, f"{mm.value} quotients differ, first x={fa.value:#x} A={fb.value:#x}"
+
+
+def test_division_fp32_random(probes):
+    mm, fa, fb = _outs()
+    assert probes.probe_div32(1 << 34, 12345, ctypes.byref(mm), ctypes.byref(fa),
+                              ctypes.byref(fb)) == 0
+    assert mm.value == 0, f"{mm.value} quotients differ, first x={fa.value:#x} A={fb.value:#x}"
+
+
+@pytest.mark.parametrize("name,expect_mode", [("nf4", 0), ("fp4", 0), ("dyn8", 0)])
+@pytest.mark.parametrize("force", [-1, 1], ids=["chosen", "bisection"])
+def test_search_exhaustive(probes, name, expect_mode, force):
+    table = TABLES[name]
+    code = code_dev(table)
+    mode = ctypes.c_int(-1)
+    mm, fa, fb = _outs()
+    assert probes.probe_search(code.data_ptr(), table.size, force, ctypes.byref(mode),
+                               ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
+    assert mode.value == expect_mode
+    assert mm.value == 0, f"{mm.value} mismatches, first xn bits {fa.value:#x} got|want {fb.value:#x}"
