@@ -118,7 +118,7 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
   constexpr int BPT = bq::kQConsumers / TPB;
   const int64_t gen_blocks = p.nb - p.full_tiles * BPT;
   int64_t want = p.full_tiles;
-  const int64_t want_gen = (gen_blocks + bq::kQConsumers / 32 - 1) / (bq::kQConsumers / 32);
+  const int64_t want_gen = (gen_blocks + bq::kQConsumerWarps - 1) / bq::kQConsumerWarps;
   if (want_gen > want) want = want_gen;
   if (want < 1) want = 1;
   const int64_t cap = static_cast<int64_t>(occ) * sms;
@@ -131,7 +131,8 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
 template <int DT, int E>
 bq_status dispatch_quantize_bs(const bq::QParams& p, const CUtensorMap& map, int dev, int sms,
                                cudaStream_t stream) {
-  constexpr int EPT = 64 / bq::ElemBytes<DT>::value;
+  // threads per quantization block: each consumer thread owns 64 bytes
+  constexpr int EPT = bq::kThreadBytes / bq::ElemBytes<DT>::value;
   switch (p.bs / EPT) {
     case 1: if constexpr (EPT == 32) return launch_quantize<DT, E, 1>(p, map, dev, sms, stream); break;
     case 2: return launch_quantize<DT, E, 2>(p, map, dev, sms, stream);

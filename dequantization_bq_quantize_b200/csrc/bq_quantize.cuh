@@ -6,39 +6,53 @@
 // (lowest index on ties), codes packed two per byte high nibble first
 // (16-entry tables) or one per byte (256-entry tables).
 //
-// Kernel design.  A persistent grid (<= 2 CTAs per SM) of 288-thread CTAs: one
+// Kernel design.  A persistent grid (2 CTAs per SM) of 288-thread CTAs: one
 // producer warp streams 16 KiB input tiles (128 rows of 128 B) into a 4-stage
 // shared-memory ring with 2-D TMA loads (128-byte swizzle, no multicast), and
 // 8 consumer warps process each tile.  Consumer thread t owns 64 contiguous
-// bytes of the tile (row t/2, half t%2), read with four conflict-free 16-byte
-// shared loads thanks to the swizzle.  A quantization block therefore spans
-// TPB = blocksize * elem_bytes / 64 consecutive threads: its absmax is a
-// shuffle-xor tree over TPB lanes, plus a shared-memory step across warps when
-// TPB > 32 (blocksize 4096 in 16-bit types, 2048+ in fp32).  The stage is
-// released right after the absmax pass (the data is in registers by then).
-// Normalisation uses the per-block reciprocal with Markstein's correction
-// (exact), the search the bucket table of bq_search.cuh, and each thread
-// stores its packed codes with one or two 16-byte stores.  Bytes of the input
-// that do not fill a whole tile, and every input that is not 16-byte aligned,
-// are handled one block per warp from global memory with the same arithmetic.
+// bytes (row t/2, half t%2), read with four conflict-free 16-byte shared
+// loads thanks to the swizzle.  A quantization block spans TPB =
+// blocksize * elem_bytes / 64 consecutive threads: its absmax is a shuffle-xor
+// tree over TPB lanes, plus a shared-memory step across warps when TPB > 32.
+// The stage is released as soon as the values are in registers.
+//
+// Per element the fast path costs about ten instructions:
+//  - 16-bit inputs: absmax from packed two-lane max of absolute values
+//    (NaN-propagating, so a block holding a NaN or inf is recognised by its
+//    absmax and takes the safe path);
+//  - xn by Markstein's correction from the block's reciprocal, two elements
+//    per instruction with the sm_100 fp32x2 FMA / MUL (no per-element range
+//    check: see div_fast);
+//  - the code from a bucket table (bq_search.cuh): one packed bucket
+//    computation per pair, two shared loads and one compare per element;
+//  - codes inserted into the output words with bit-field inserts.
+// Blocks whose absmax is outside [2^-60, 2^60] (or not finite), and codebooks
+// without a bucket table, take the safe path: IEEE division where Markstein's
+// form is not valid, and a clamped lookup.  Bytes of the input that do not
+// fill a whole tile, and every input that is not 16-byte aligned, are handled
+// one block per warp from global memory with IEEE division.
 #pragma once
 
 #include "bq_search.cuh"
 
 namespace bq {
 
-constexpr int kQThreads = 288;    // warp 0: producer; warps 1..8: consumers
-constexpr int kQConsumers = 256;
+constexpr int kQConsumerWarps = 8;
+constexpr int kQConsumers = kQConsumerWarps * 32;  // 256
+constexpr int kQThreads = kQConsumers + 32;        // + producer warp
 constexpr int kTileBytes = 16384;
-constexpr int kTileRows = 128;    // rows of 128 bytes
+constexpr int kTileRows = 128;                     // rows of 128 bytes
 constexpr int kStages = 4;
+constexpr int kThreadBytes = kTileBytes / kQConsumers;  // 64
+constexpr int kThreadWords = kThreadBytes / 4;           // 16
+static_assert(kThreadBytes == 64, "thread owns four 16-byte chunks");
 
 template <int E>
 struct QSmem {
   uint8_t stage[kStages][kTileBytes];  // 1024-byte aligned (128B swizzle)
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  float red[2][8];
+  float red[2][kQConsumerWarps];
   int cabort[2];   // per tile-iteration parity: a consumer gave up waiting
   TableSmem tab;
   Lut<E> lut;
@@ -58,53 +72,151 @@ struct QParams {
   int32_t bs;
 };
 
-// ------------------------------------------------- one element -> code ----
+// ------------------------------------------------------ small helpers -----
 
-template <int DT, int EPT>
-__device__ __forceinline__ float tile_elem(const uint32_t (&w)[16], int j) {
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// Packed two-lane |a| vs |b| max (NaN-propagating) and min; the sign of the
+// result is meaningless and dropped later.
+template <int DT>
+__device__ __forceinline__ uint32_t amax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  if constexpr (DT == kBF16) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  else asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <int DT>
+__device__ __forceinline__ uint32_t amin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  if constexpr (DT == kBF16) asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  else asm("min.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bfi(uint32_t field, uint32_t base, int pos, int len) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(field), "r"(base), "r"(pos), "r"(len));
+  return d;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+template <int DT>
+__device__ __forceinline__ float tile_elem(const uint32_t (&w)[kThreadWords], int j) {
   if constexpr (DT == kF32) return __uint_as_float(w[j]);
   else return widen_pair_elem<DT>(w[j >> 1], j & 1);
 }
 
-// Codes of a thread's EPT elements packed into words: 4-bit codes put element
-// 2i in the high nibble of byte i; 8-bit codes one per byte.
-template <int DT, int E, int MODE, int EPT, bool SLOW>
-__device__ __forceinline__ void encode_thread(const uint32_t (&w)[16], const BlockScale& sc,
-                                              const TableSmem& tab, const Lut<E>& lut,
-                                              uint32_t (&ow)[E == 16 ? EPT / 8 : EPT / 4],
-                                              bool& any_small) {
-  constexpr int NW = E == 16 ? EPT / 8 : EPT / 4;
-#pragma unroll
-  for (int k = 0; k < NW; ++k) ow[k] = 0;
-  bool small = false;
-#pragma unroll
-  for (int j = 0; j < EPT; ++j) {
-    const float x = tile_elem<DT, EPT>(w, j);
-    float xn;
-    if constexpr (SLOW) {
-      xn = fabsf(x) < sc.theta ? div_exact(x, sc.A) : div_fast(x, sc);
-    } else {
-      xn = div_fast(x, sc);
-      if constexpr (DT != kF16) small |= fabsf(x) < sc.theta;
-    }
-    const uint32_t c = search<E, MODE>(xn, tab, lut);
-    if constexpr (E == 16) {
-      ow[j >> 3] |= c << ((((j & 7) >> 1) << 3) + ((j & 1) ? 0 : 4));
-    } else {
-      ow[j >> 2] |= c << ((j & 3) << 3);
-    }
+// Output bit position of element j in the thread's code words.
+template <int E>
+__device__ __forceinline__ constexpr int code_pos(int j) {
+  if constexpr (E == 16) return (((j & 7) >> 1) << 3) + ((j & 1) ? 0 : 4);
+  else return (j & 3) << 3;
+}
+
+// Codes of one thread: EPT elements -> OUT_BYTES bytes in NW words.
+template <int DT, int E>
+struct QOut {
+  static constexpr int EPT = kThreadBytes / ElemBytes<DT>::value;
+  static constexpr int BYTES = E == 16 ? EPT / 2 : EPT;
+  static constexpr int NW = BYTES / 4;
+  static constexpr int L = E == 16 ? 4 : 8;        // bits per code
+  static constexpr int PER_WORD = 32 / L;
+};
+
+// ------------------------------------------------------ fast encoding -----
+
+// Shared address of lut.t[bucket].  For 16-entry tables `b` is already
+// fma(xn, 15, 1.5 * 2^23) and t_base = &lut.t[0] - 4 * (0x4B400000 - 15), so
+// bits(b) * 4 + t_base addresses the bucket (32-bit wrap-around arithmetic).
+// For 256-entry tables b is xn and t_base = &lut.t[1537].
+template <int E>
+__device__ __forceinline__ uint32_t lut_addr(float b, uint32_t t_base) {
+  if constexpr (E == 16) {
+    return __float_as_uint(b) * 4u + t_base;
+  } else {
+    const uint32_t u = __float_as_uint(b);
+    const uint32_t a = u & 0x7fffffffu;
+    const uint32_t idx = (max(a, 0x33800000u) - 0x33800000u) >> 17;
+    const uint32_t sgn = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31);
+    return (idx ^ sgn) * 4u + t_base;
   }
-  any_small = small;
+}
+
+template <int E>
+__device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut) {
+  if constexpr (E == 16) return smem_u32(lut.t) - 4u * (0x4B400000u - 15u);
+  else return smem_u32(lut.t) + 4u * 1537u;
+}
+
+// Fast path: finite block, every |x| large enough for Markstein's form, and a
+// bucket table.  Two elements per packed division and bucket computation.
+template <int DT, int E>
+__device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
+                                            uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
+  using O = QOut<DT, E>;
+  constexpr uint32_t CW_OFF = 4u * LutSize<E>::value;  // lut.cw follows lut.t
+#pragma unroll
+  for (int k = 0; k < O::NW; ++k) ow[k] = 0u;
+#pragma unroll
+  for (int i = 0; i < O::EPT / 2; ++i) {
+    float q0, q1;
+    div_fast2(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
+    float b0 = q0, b1 = q1;
+    if constexpr (E == 16)
+      unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
+    const uint32_t a0 = lut_addr<E>(b0, t_base), a1 = lut_addr<E>(b1, t_base);
+    const float t0 = lds_f32(a0), t1 = lds_f32(a1);
+    const uint32_t w0 = lds_u32(a0 + CW_OFF), w1 = lds_u32(a1 + CW_OFF);
+    const uint32_t c0 = q0 >= t0 ? (w0 >> 8) : w0;
+    const uint32_t c1 = q1 >= t1 ? (w1 >> 8) : w1;
+    const int j0 = 2 * i, j1 = 2 * i + 1;
+    ow[j0 / O::PER_WORD] = bfi(c0, ow[j0 / O::PER_WORD], code_pos<E>(j0), O::L);
+    ow[j1 / O::PER_WORD] = bfi(c1, ow[j1 / O::PER_WORD], code_pos<E>(j1), O::L);
+  }
+}
+
+// Any table form, any block: IEEE division where Markstein's form is not
+// valid, clamped lookups.  Exact for every finite input, and never indexes
+// outside the tables for any input.  Inlined (an out-of-line call would move
+// the thread's registers through local memory on every tile).
+template <int DT, int E, int MODE>
+__device__ __forceinline__ void encode_safe(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
+                                            const TableSmem& tab, const Lut<E>& lut,
+                                            uint32_t (&ow)[QOut<DT, E>::NW]) {
+  using O = QOut<DT, E>;
+#pragma unroll
+  for (int k = 0; k < O::NW; ++k) ow[k] = 0u;
+#pragma unroll
+  for (int j = 0; j < O::EPT; ++j) {
+    const float x = tile_elem<DT>(w, j);
+    const float xn = fabsf(x) < sc.theta ? div_exact(x, sc.A) : div_fast(x, sc);
+    const uint32_t c = search<E, MODE>(xn, tab, lut);
+    ow[j / O::PER_WORD] |= (c & ((1u << O::L) - 1u)) << code_pos<E>(j);
+  }
 }
 
 // --------------------------------------------------- one tile (consumer) --
 
 template <int DT, int E, int TPB, int MODE>
-__device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, int64_t tile,
-                                              int st, uint32_t par, int64_t iter, int ct) {
-  constexpr int EB = ElemBytes<DT>::value;
-  constexpr int EPT = 64 / EB;
-  constexpr int TE = kTileBytes / EB;
+__device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uint32_t tile,
+                                              int st, uint32_t par, uint32_t iter, int ct,
+                                              uint32_t t_base) {
+  using O = QOut<DT, E>;
+  constexpr int TE = kTileBytes / ElemBytes<DT>::value;
   constexpr int BPT = kQConsumers / TPB;
   const int lane = ct & 31, cw = ct >> 5;
 
@@ -115,7 +227,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, int
   }
 
   // four 16-byte chunks of row ct/2, physical chunk = logical ^ (row % 8)
-  uint32_t w[16];
+  uint32_t w[kThreadWords];
   {
     const int r = ct >> 1;
     const uint8_t* row = s.stage[st] + r * 128;
@@ -126,19 +238,30 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, int
       w[4 * k + 0] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
     }
   }
-  float m = 0.0f;
+
+  // thread-local absmax, NaN-propagating
+  float amax;
+  if constexpr (DT == kF32) {
+    amax = fabsf(__uint_as_float(w[0]));
 #pragma unroll
-  for (int j = 0; j < EPT; ++j) m = fmaxf(m, fabsf(tile_elem<DT, EPT>(w, j)));
+    for (int j = 1; j < kThreadWords; ++j) amax = max_nan(amax, fabsf(__uint_as_float(w[j])));
+  } else {
+    uint32_t m2 = amax2<DT>(w[0], w[1]);
+#pragma unroll
+    for (int j = 2; j < kThreadWords; ++j) m2 = amax2<DT>(m2, w[j]);
+    amax = max_nan(fabsf(widen_pair_elem<DT>(m2, 0)), fabsf(widen_pair_elem<DT>(m2, 1)));
+  }
   __syncwarp();
   if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
 
   bool abort_now = !ok;
+  float m = amax;
   if constexpr (TPB > 1 && TPB <= 32) {
 #pragma unroll
-    for (int off = 1; off < TPB; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int off = 1; off < TPB; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
   } else if constexpr (TPB > 32) {
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int off = 1; off < 32; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
     constexpr int WPB = TPB / 32;
     const int pb = static_cast<int>(iter & 1);
     if (lane == 0) s.red[pb][cw] = m;
@@ -146,7 +269,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, int
     const int g0 = (cw / WPB) * WPB;
     m = s.red[pb][g0];
 #pragma unroll
-    for (int i = 1; i < WPB; ++i) m = fmaxf(m, s.red[pb][g0 + i]);
+    for (int i = 1; i < WPB; ++i) m = max_nan(m, s.red[pb][g0 + i]);
     // set before this barrier by any warp that gave up on this tile; the slot
     // of the other parity may already be written by a warp one tile ahead
     abort_now = *reinterpret_cast<volatile int*>(&s.cabort[iter & 1]) != 0;
@@ -154,24 +277,25 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, int
   const float A = m;
   if (abort_now) return false;
 
-  const int64_t e0 = tile * TE + static_cast<int64_t>(ct) * EPT;
-  if (ct % TPB == 0) p.absmax[tile * BPT + ct / TPB] = A;
+  if (ct % TPB == 0) p.absmax[static_cast<int64_t>(tile) * BPT + ct / TPB] = A;
 
   const BlockScale sc = make_scale(A);
-  constexpr int NW = E == 16 ? EPT / 8 : EPT / 4;
-  uint32_t ow[NW];
-  bool any_small;
-  encode_thread<DT, E, MODE, EPT, false>(w, sc, s.tab, s.lut, ow, any_small);
-  if (any_small) encode_thread<DT, E, MODE, EPT, true>(w, sc, s.tab, s.lut, ow, any_small);
+  uint32_t ow[O::NW];
+  // bucket path: the block's reciprocal is valid for Markstein's form (the
+  // per-element condition is not needed, see div_fast); NaN fails both tests
+  const bool fast = MODE == kModeLut && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
+  if (fast) encode_fast<DT, E>(w, sc, t_base, ow);
+  else encode_safe<DT, E, MODE>(w, sc, s.tab, s.lut, ow);
 
+  const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
   uint8_t* dst = p.out + (E == 16 ? e0 / 2 : e0);
-  if constexpr (NW == 2) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(ow[0], ow[1]);
-  } else {
 #pragma unroll
-    for (int k = 0; k < NW; k += 4)
+  for (int k = 0; k < O::NW; k += 4) {
+    if constexpr (O::NW >= 4) {
       *reinterpret_cast<uint4*>(dst + 4 * k) = make_uint4(ow[k], ow[k + 1], ow[k + 2], ow[k + 3]);
+    }
   }
+  if constexpr (O::NW == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(ow[0], ow[1]);
   return true;
 }
 
@@ -182,9 +306,9 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
   const int64_t lo = b * p.bs;
   const int64_t hi = min(p.n, lo + p.bs);
   float m = 0.0f;
-  for (int64_t i = lo + lane; i < hi; i += 32) m = fmaxf(m, fabsf(load_elem<DT>(p.x, i)));
+  for (int64_t i = lo + lane; i < hi; i += 32) m = max_nan(m, fabsf(load_elem<DT>(p.x, i)));
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = 16; off >= 1; off >>= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
   const float A = m;
   if (lane == 0) p.absmax[b] = A;
   if constexpr (E == 16) {
@@ -193,7 +317,7 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
       const uint32_t c0 = search<E, MODE>(div_exact(load_elem<DT>(p.x, i0), A), s.tab, s.lut);
       uint32_t c1 = 0;
       if (i0 + 1 < hi) c1 = search<E, MODE>(div_exact(load_elem<DT>(p.x, i0 + 1), A), s.tab, s.lut);
-      p.out[q] = static_cast<uint8_t>((c0 << 4) | c1);
+      p.out[q] = static_cast<uint8_t>(((c0 & 15u) << 4) | (c1 & 15u));
     }
   } else {
     for (int64_t i = lo + lane; i < hi; i += 32)
@@ -205,19 +329,19 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 
 template <int DT, int E, int TPB, int MODE>
 __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int ct) {
-  constexpr int EB = ElemBytes<DT>::value;
   constexpr int BPT = kQConsumers / TPB;
-  int64_t iter = 0;
-  for (int64_t tile = blockIdx.x; tile < p.full_tiles; tile += gridDim.x, ++iter) {
+  const uint32_t t_base = lut_base<E>(s.lut);
+  const uint32_t ntiles = static_cast<uint32_t>(p.full_tiles);  // < 2^24 (host check)
+  uint32_t iter = 0;
+  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
     const int st = static_cast<int>(iter % kStages);
-    const uint32_t par = static_cast<uint32_t>((iter / kStages) & 1);
-    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct)) break;
+    const uint32_t par = (iter / kStages) & 1u;
+    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base)) break;
   }
-  (void)EB;
   // what the tiles did not cover: one quantization block per warp
   const int lane = ct & 31, cw = ct >> 5;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kQConsumers / 32);
-  for (int64_t b = p.full_tiles * BPT + static_cast<int64_t>(blockIdx.x) * (kQConsumers / 32) + cw;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kQConsumerWarps;
+  for (int64_t b = p.full_tiles * BPT + static_cast<int64_t>(blockIdx.x) * kQConsumerWarps + cw;
        b < p.nb; b += nwarps)
     quantize_block_generic<DT, E, MODE>(p, s, b, lane);
 }
@@ -233,7 +357,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kQConsumers / 32);
+      mbar_init(&s.empty[i], kQConsumerWarps);
     }
     s.cabort[0] = 0;
     s.cabort[1] = 0;
@@ -264,7 +388,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
   }
 
   const int ct = threadIdx.x - 32;
-  build_search<E>(s.tab, s.lut, p.code, ct);
+  build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   const int mode = s.tab.mode;
   if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);
   else if (mode == kModeBsearch) consumer_main<DT, E, TPB, kModeBsearch>(s, p, ct);

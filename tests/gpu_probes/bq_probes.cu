@@ -26,9 +26,27 @@ __device__ __forceinline__ bool same_quotient(float a, float b) {
   return __float_as_uint(a) == __float_as_uint(b) || (a == 0.0f && b == 0.0f);
 }
 
-__device__ __forceinline__ float kernel_division(float x, float A) {
+// The quantize kernels' bucket path divides elements in pairs with the packed
+// Markstein form (div_fast2) for every block whose absmax is in [2^-60, 2^60],
+// without a per-element check: it needs the exact quotient, except that when
+// the exact quotient is below 2^-38 in magnitude the result only has to be
+// below 2^-38 too.  The safe path uses IEEE division for |x| < A 2^-40.
+// Both are checked; the packed form on both lanes (the second with -x).
+__device__ __forceinline__ bool bucket_path_ok(float got, float want) {
+  return same_quotient(got, want) || (fabsf(got) < 0x1p-38f && fabsf(want) < 0x1p-38f);
+}
+
+__device__ __forceinline__ bool division_ok(float x, float A) {
   const bq::BlockScale s = bq::make_scale(A);
-  return fabsf(x) < s.theta ? bq::div_exact(x, A) : bq::div_fast(x, s);
+  const float w0 = __fdiv_rn(x, A), w1 = __fdiv_rn(-x, A);
+  bool ok = true;
+  if (A >= 0x1p-60f && A <= 0x1p60f) {
+    float q0, q1;
+    bq::div_fast2(x, -x, s, q0, q1);
+    ok = bucket_path_ok(q0, w0) && bucket_path_ok(q1, w1);
+  }
+  const float safe = fabsf(x) < s.theta ? bq::div_exact(x, A) : bq::div_fast(x, s);
+  return ok && same_quotient(safe, w0);
 }
 
 __device__ void report(unsigned int a, unsigned int b) {
@@ -47,9 +65,7 @@ __global__ void div16_all(int a_lo) {
   for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
     const float x = bq::widen_pair_elem<DT>(xb, 0);
     if (!isfinite(x) || !(fabsf(x) <= A)) continue;
-    const float got = kernel_division(x, A);
-    const float want = __fdiv_rn(x, A);
-    if (!same_quotient(got, want)) report(xb, a_bits);
+    if (!division_ok(x, A)) report(xb, a_bits);
   }
 }
 
@@ -74,9 +90,7 @@ __global__ void div32_random(uint64_t count, uint64_t seed) {
     float x = __uint_as_float(xb);
     if (!isfinite(A) || !isfinite(x) || A == 0.0f) continue;
     if (fabsf(x) > A) { const float t = A; A = fabsf(x); x = copysignf(t, x); }
-    const float got = kernel_division(x, A);
-    const float want = __fdiv_rn(x, A);
-    if (!same_quotient(got, want)) report(__float_as_uint(x), __float_as_uint(A));
+    if (!division_ok(x, A)) report(__float_as_uint(x), __float_as_uint(A));
   }
 }
 
@@ -106,7 +120,7 @@ __global__ void __launch_bounds__(256) search_all(const float* code, int* mode_o
   extern __shared__ uint8_t raw[];
   ProbeSmem<E>& s = *reinterpret_cast<ProbeSmem<E>*>(raw);
   const int ct = threadIdx.x;
-  bq::build_search<E>(s.tab, s.lut, code, ct);
+  bq::build_search<E, 256>(s.tab, s.lut, code, ct);
   if (ct < E) s.c[ct] = code[ct];
   __syncthreads();
   const int mode = s.tab.mode;
@@ -133,7 +147,7 @@ __global__ void __launch_bounds__(256) search_forced(const float* code, int* mod
   extern __shared__ uint8_t raw[];
   ProbeSmem<E>& s = *reinterpret_cast<ProbeSmem<E>*>(raw);
   const int ct = threadIdx.x;
-  bq::build_search<E>(s.tab, s.lut, code, ct);
+  bq::build_search<E, 256>(s.tab, s.lut, code, ct);
   if (ct < E) s.c[ct] = code[ct];
   __syncthreads();
   if (blockIdx.x == 0 && ct == 0) *mode_out = s.tab.mode;
@@ -148,6 +162,27 @@ __global__ void __launch_bounds__(256) search_forced(const float* code, int* mod
     const uint32_t got = bq::search<E, MODE>(xn, s.tab, s.lut);
     const uint32_t want = plain_scan<E>(xn, s.c);
     if (got != want) report(bits, (got << 16) | want);
+  }
+}
+
+// ------------------------------------------------------- bounded wait ----
+
+// One thread waits on an mbarrier that nothing ever arrives on.  The wait must
+// give up by itself (bounded by bq::kWaitLimitNs) and report it; the context
+// stays usable afterwards.
+__global__ void wait_timeout(int* result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    bq::mbar_init(&bar, 1);
+    bq::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = bq::globaltimer_ns();
+    const bool ok = bq::mbar_wait_bounded(&bar, 0);
+    const uint64_t t1 = bq::globaltimer_ns();
+    result[0] = ok ? 1 : 0;
+    result[1] = static_cast<int>((t1 - t0) / 1000000ull);
   }
 }
 
@@ -234,6 +269,19 @@ __attribute__((visibility("default"))) int probe_search(const float* code, int e
   if (mode_request == 1)
     return run_search<256>(search_forced<256, bq::kModeBsearch>, code, mode_out, mm, fa, fb);
   return run_search<256>(search_all<256>, code, mode_out, mm, fa, fb);
+}
+
+// result[0] = 1 if the wait completed (it must not), result[1] = ms waited.
+__attribute__((visibility("default"))) int probe_wait_timeout(int* result) {
+  int* d = nullptr;
+  cudaError_t e = cudaMalloc(&d, 2 * sizeof(int));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  wait_timeout<<<1, 32>>>(d);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(result, d, 2 * sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  return static_cast<int>(e);
 }
 
 }  // extern "C"

@@ -340,6 +340,7 @@ def probes():
     L.probe_div32.argtypes = [ctypes.c_ulonglong, ctypes.c_ulonglong, u64p, u32p, u32p]
     L.probe_search.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                ctypes.POINTER(ctypes.c_int), u64p, u32p, u32p]
+    L.probe_wait_timeout.argtypes = [ctypes.POINTER(ctypes.c_int)]
     return L
 
 
@@ -372,3 +373,15 @@ def test_search_exhaustive(probes, name, expect_mode, force):
                                ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
     assert mode.value == expect_mode
     assert mm.value == 0, f"{mm.value} mismatches, first xn bits {fa.value:#x} got|want {fb.value:#x}"
+
+
+def test_bounded_wait_gives_up_and_context_survives(probes):
+    """An mbarrier wait that nothing completes returns 'timed out' after the
+    library's limit (about 2 s) instead of hanging; the GPU stays usable."""
+    res = (ctypes.c_int * 2)(-1, -1)
+    assert probes.probe_wait_timeout(res) == 0
+    assert res[0] == 0, "the wait claims to have completed"
+    assert 1500 <= res[1] <= 10000, f"gave up after {res[1]} ms"
+    # the context is still healthy: a normal quantize call works
+    x = small_input(8192 * 2 + 5, "bf16", 64, seed=1)
+    check_quant(x, "bf16", 64, "nf4")
