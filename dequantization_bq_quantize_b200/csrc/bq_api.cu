@@ -190,8 +190,8 @@ bq_status launch_gguf(const bq::GParams& p, int dev, int sms, cudaStream_t strea
   int occ = 1;
   bq_status s = kernel_occupancy(slot, kernel, dev, bq::kGThreads, 0, &occ);
   if (s != BQ_OK) return s;
-  const int64_t groups = (p.n_blocks + bq::kGGroup - 1) / bq::kGGroup;
-  int64_t want = (groups + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
+  const int64_t steps = (p.n_blocks + bq::kGGroup * bq::kGUnroll - 1) / (bq::kGGroup * bq::kGUnroll);
+  int64_t want = (steps + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   if (want > cap) want = cap;
   if (want < 1) want = 1;

@@ -82,6 +82,29 @@ __device__ __forceinline__ void store_elem(void* y, int64_t i, float v) {
   }
 }
 
+// ------------------------------------------------ packed fp32 pairs ------
+
+// Two fp32 lanes in one 64-bit register: the sm_100 f32x2 instructions do two
+// IEEE operations (round to nearest even, no flush) per instruction.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // ------------------------------------------------------------ PTX wrappers --
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

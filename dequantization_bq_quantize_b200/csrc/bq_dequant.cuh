@@ -9,13 +9,17 @@
 // 16-bit type, 4 of fp32); one thread makes one chunk, so every warp-wide
 // store is 512 contiguous bytes and every warp-wide code load is contiguous
 // too.  A chunk never straddles a quantization block (blocksize >= 32), so it
-// needs one absmax.  Each thread handles four chunks a grid-stride apart per
-// iteration with all loads issued first.  Buffers that are not aligned for the
-// vector path, and the elements after the last whole chunk, are done one
-// element per thread.
+// needs one absmax.  Each thread handles eight chunks a grid-stride apart per
+// iteration with all loads issued first.
+// 4-bit codes: a byte holds the codes of two neighbouring elements, so the
+// shared table is indexed by the whole byte and holds the pair
+// (code[byte >> 4], code[byte & 15]): one 64-bit shared load and one packed
+// fp32x2 multiply per two elements.  8-bit codes: one 32-bit load per element,
+// multiplied in pairs.  Buffers that are not aligned for the vector path, and
+// the elements after the last whole chunk, are done one element per thread.
 #pragma once
 
-#include "bq_common.cuh"
+#include "bq_search.cuh"
 
 namespace bq {
 
@@ -31,12 +35,20 @@ struct DParams {
 };
 
 constexpr int kDThreads = 256;
+constexpr int kDUnroll = 8;
 
 template <int E, int OT>
 struct DTraits {
   static constexpr int OB = OT == kF32 ? 4 : 2;       // output element bytes
   static constexpr int CE = 16 / OB;                  // elements per chunk
   static constexpr int QB = E == 16 ? CE / 2 : CE;    // code bytes per chunk
+};
+
+template <int E>
+struct DSmem {
+  // E == 16: pair[b] = (code[b >> 4], code[b & 15]); E == 256: code[b]
+  float t[E == 16 ? 512 : 256];
+  float code[E];
 };
 
 template <int QB>
@@ -50,24 +62,37 @@ __device__ __forceinline__ uint2 load_codes(const uint8_t* __restrict__ q, int64
   }
 }
 
-// Code index of element e (0..CE-1) of a chunk whose code bytes are in c.
+// Two outputs from one code byte pair index / two code bytes, times A.  The
+// table reads are asm with no memory dependence: their addresses come from
+// code bytes loaded from global memory after the table was built and
+// __syncthreads, and that data dependence keeps them after the build.
 template <int E>
-__device__ __forceinline__ uint32_t chunk_code(uint2 c, int e) {
+__device__ __forceinline__ void decode_pair(uint2 c, int k, uint32_t t_base, uint64_t a2,
+                                            float& v0, float& v1) {
   if constexpr (E == 16) {
-    const uint32_t byte = (c.x >> ((e >> 1) << 3)) & 0xffu;
-    return (e & 1) ? (byte & 15u) : (byte >> 4);
+    // byte k of the chunk's code word: elements 2k (high nibble), 2k+1 (low)
+    const uint32_t byte = __byte_perm(c.x, 0u, 0x4440u + k);
+    uint2 pr;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(pr.x), "=r"(pr.y) : "r"(t_base + byte * 8u));
+    unpack2(mul2(pack2(__uint_as_float(pr.x), __uint_as_float(pr.y)), a2), v0, v1);
   } else {
-    const uint32_t word = e < 4 ? c.x : c.y;
-    return (word >> ((e & 3) << 3)) & 0xffu;
+    const uint32_t word = k < 2 ? c.x : c.y;
+    const uint32_t b0 = __byte_perm(word, 0u, 0x4440u + 2 * (k & 1));
+    const uint32_t b1 = __byte_perm(word, 0u, 0x4441u + 2 * (k & 1));
+    float c0, c1;
+    asm("ld.shared.f32 %0, [%1];" : "=f"(c0) : "r"(t_base + b0 * 4u));
+    asm("ld.shared.f32 %0, [%1];" : "=f"(c1) : "r"(t_base + b1 * 4u));
+    unpack2(mul2(pack2(c0, c1), a2), v0, v1);
   }
 }
 
 template <int E, int OT>
-__device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, const float* sc) {
+__device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, uint32_t t_base) {
   constexpr int CE = DTraits<E, OT>::CE;
+  const uint64_t a2 = pack2(A, A);
   float v[CE];
 #pragma unroll
-  for (int e = 0; e < CE; ++e) v[e] = __fmul_rn(sc[chunk_code<E>(c, e)], A);
+  for (int k = 0; k < CE / 2; ++k) decode_pair<E>(c, k, t_base, a2, v[2 * k], v[2 * k + 1]);
   if constexpr (OT == kF32) {
     return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
                       __float_as_uint(v[3]));
@@ -79,16 +104,26 @@ __device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, const float* sc)
 
 template <int E, int OT>
 __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
-  __shared__ float sc[E];
-  for (int i = threadIdx.x; i < E; i += blockDim.x) sc[i] = p.code[i];
+  __shared__ DSmem<E> s;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) s.code[i] = p.code[i];
   __syncthreads();
+  if constexpr (E == 16) {
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+      s.t[2 * b] = s.code[b >> 4];
+      s.t[2 * b + 1] = s.code[b & 15];
+    }
+  } else {
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) s.t[b] = s.code[b];
+  }
+  __syncthreads();
+  const uint32_t t_base = smem_u32(s.t);
 
   using T = DTraits<E, OT>;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t gsz = static_cast<int64_t>(gridDim.x) * blockDim.x;
 
   if (p.vec) {
-    constexpr int U = 4;
+    constexpr int U = kDUnroll;
     uint4* y4 = static_cast<uint4*>(p.y);
     for (int64_t base = gtid; base < p.nchunks; base += U * gsz) {
       uint2 c[U];
@@ -104,7 +139,7 @@ __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t ch = base + u * gsz;
-        if (ch < p.nchunks) y4[ch] = decode_chunk<E, OT>(c[u], A[u], sc);
+        if (ch < p.nchunks) y4[ch] = decode_chunk<E, OT>(c[u], A[u], t_base);
       }
     }
   }
@@ -118,7 +153,7 @@ __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
     } else {
       idx = p.q[i];
     }
-    store_elem<OT>(p.y, i, __fmul_rn(sc[idx], p.absmax[i >> p.bs_log2]));
+    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], p.absmax[i >> p.bs_log2]));
   }
 }
 

@@ -103,14 +103,13 @@ __device__ __forceinline__ uint32_t bfi(uint32_t field, uint32_t base, int pos, 
   return d;
 }
 
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+// Table read by shared-window address.  The asm has no memory dependence, so
+// it is only ever fed addresses computed from tile data loaded after the
+// mbarrier wait (itself after the table build and its barrier): the data
+// dependence keeps it after both.
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
@@ -139,36 +138,58 @@ struct QOut {
 
 // ------------------------------------------------------ fast encoding -----
 
-// Shared address of lut.t[bucket].  For 16-entry tables `b` is already
-// fma(xn, 15, 1.5 * 2^23) and t_base = &lut.t[0] - 4 * (0x4B400000 - 15), so
-// bits(b) * 4 + t_base addresses the bucket (32-bit wrap-around arithmetic).
-// For 256-entry tables b is xn and t_base = &lut.t[1537].
+// Shared address of lut.e[bucket].  For 16-entry tables `b` is already
+// fma(xn, 15, 1.5 * 2^23) and t_base = &lut.e[0] - 8 * (0x4B400000 - 15), so
+// bits(b) * 8 + t_base addresses the bucket (32-bit wrap-around arithmetic).
+// For 256-entry tables b is xn and t_base = &lut.e[1537].
 template <int E>
 __device__ __forceinline__ uint32_t lut_addr(float b, uint32_t t_base) {
   if constexpr (E == 16) {
-    return __float_as_uint(b) * 4u + t_base;
+    return __float_as_uint(b) * 8u + t_base;
   } else {
     const uint32_t u = __float_as_uint(b);
     const uint32_t a = u & 0x7fffffffu;
     const uint32_t idx = (max(a, 0x33800000u) - 0x33800000u) >> 17;
     const uint32_t sgn = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31);
-    return (idx ^ sgn) * 4u + t_base;
+    return (idx ^ sgn) * 8u + t_base;
   }
 }
 
 template <int E>
 __device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut) {
-  if constexpr (E == 16) return smem_u32(lut.t) - 4u * (0x4B400000u - 15u);
-  else return smem_u32(lut.t) + 4u * 1537u;
+  if constexpr (E == 16) return smem_u32(lut.e) - 8u * (0x4B400000u - 15u);
+  else return smem_u32(lut.e) + 8u * 1537u;
 }
 
-// Fast path: finite block, every |x| large enough for Markstein's form, and a
-// bucket table.  Two elements per packed division and bucket computation.
-template <int DT, int E>
+// Weight of element j within its 16-bit half of the output: a half holds 4
+// codes of 4 bits (element order in a byte: high nibble first) or 2 codes of
+// 8 bits, little-endian.
+template <int E>
+__device__ __forceinline__ constexpr float half_weight(int j) {
+  if constexpr (E == 16) {
+    constexpr float w4[4] = {16.0f, 1.0f, 4096.0f, 256.0f};
+    return w4[j & 3];
+  } else {
+    return (j & 1) ? 256.0f : 1.0f;
+  }
+}
+
+// Fast path: the block's reciprocal is valid for Markstein's form and the
+// codebook has a bucket table.  Two elements per packed division and bucket
+// computation; one 64-bit table load per element.
+//  kModeLut:  code = q >= t ? code1 : code0, inserted with a bit-field insert.
+//  kModeLutF: H = sat(fma(q, 2^60, K)) is exactly [q >= t]; code = C + H is
+//             accumulated in fp32 into 16-bit halves (2^23 + sum of
+//             code * weight, every value an exact integer below 2^24; the
+//             first element of a half brings the 2^23), and the halves' low
+//             bytes are merged with one byte permute per word.
+template <int DT, int E, int MODE>
 __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
                                             uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
   using O = QOut<DT, E>;
-  constexpr uint32_t CW_OFF = 4u * LutSize<E>::value;  // lut.cw follows lut.t
+  constexpr int NH = 2 * O::NW;                 // 16-bit halves
+  constexpr int PER_HALF = O::EPT / NH;         // elements per half (4 or 2)
+  float hacc[NH];
 #pragma unroll
   for (int k = 0; k < O::NW; ++k) ow[k] = 0u;
 #pragma unroll
@@ -178,14 +199,30 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
     float b0 = q0, b1 = q1;
     if constexpr (E == 16)
       unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
-    const uint32_t a0 = lut_addr<E>(b0, t_base), a1 = lut_addr<E>(b1, t_base);
-    const float t0 = lds_f32(a0), t1 = lds_f32(a1);
-    const uint32_t w0 = lds_u32(a0 + CW_OFF), w1 = lds_u32(a1 + CW_OFF);
-    const uint32_t c0 = q0 >= t0 ? (w0 >> 8) : w0;
-    const uint32_t c1 = q1 >= t1 ? (w1 >> 8) : w1;
+    const uint2 e0 = lds_u64(lut_addr<E>(b0, t_base));
+    const uint2 e1 = lds_u64(lut_addr<E>(b1, t_base));
     const int j0 = 2 * i, j1 = 2 * i + 1;
-    ow[j0 / O::PER_WORD] = bfi(c0, ow[j0 / O::PER_WORD], code_pos<E>(j0), O::L);
-    ow[j1 / O::PER_WORD] = bfi(c1, ow[j1 / O::PER_WORD], code_pos<E>(j1), O::L);
+    if constexpr (MODE == kModeLutF) {
+      const float h0 = fma_sat(q0, kSelScale, __uint_as_float(e0.x));
+      const float h1 = fma_sat(q1, kSelScale, __uint_as_float(e1.x));
+      float& a0 = hacc[j0 / PER_HALF];
+      a0 = __fmaf_rn(__uint_as_float(e0.y), half_weight<E>(j0),
+                     j0 % PER_HALF == 0 ? 8388608.0f : a0);  // 2^23 enters once
+      a0 = __fmaf_rn(h0, half_weight<E>(j0), a0);
+      float& a1 = hacc[j1 / PER_HALF];
+      a1 = __fmaf_rn(__uint_as_float(e1.y), half_weight<E>(j1), a1);
+      a1 = __fmaf_rn(h1, half_weight<E>(j1), a1);
+    } else {
+      const uint32_t c0 = q0 >= __uint_as_float(e0.x) ? (e0.y >> 8) : e0.y;
+      const uint32_t c1 = q1 >= __uint_as_float(e1.x) ? (e1.y >> 8) : e1.y;
+      ow[j0 / O::PER_WORD] = bfi(c0, ow[j0 / O::PER_WORD], code_pos<E>(j0), O::L);
+      ow[j1 / O::PER_WORD] = bfi(c1, ow[j1 / O::PER_WORD], code_pos<E>(j1), O::L);
+    }
+  }
+  if constexpr (MODE == kModeLutF) {
+#pragma unroll
+    for (int k = 0; k < O::NW; ++k)
+      ow[k] = __byte_perm(__float_as_uint(hacc[2 * k]), __float_as_uint(hacc[2 * k + 1]), 0x5410);
   }
 }
 
@@ -279,13 +316,13 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
 
   if (ct % TPB == 0) p.absmax[static_cast<int64_t>(tile) * BPT + ct / TPB] = A;
 
-  const BlockScale sc = make_scale(A);
   uint32_t ow[O::NW];
   // bucket path: the block's reciprocal is valid for Markstein's form (the
   // per-element condition is not needed, see div_fast); NaN fails both tests
-  const bool fast = MODE == kModeLut && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
-  if (fast) encode_fast<DT, E>(w, sc, t_base, ow);
-  else encode_safe<DT, E, MODE>(w, sc, s.tab, s.lut, ow);
+  constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
+  const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
+  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, ow);
+  else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
   uint8_t* dst = p.out + (E == 16 ? e0 / 2 : e0);
@@ -390,7 +427,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
   const int ct = threadIdx.x - 32;
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   const int mode = s.tab.mode;
-  if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);
+  if (mode == kModeLutF) consumer_main<DT, E, TPB, kModeLutF>(s, p, ct);
+  else if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);
   else if (mode == kModeBsearch) consumer_main<DT, E, TPB, kModeBsearch>(s, p, ct);
   else consumer_main<DT, E, TPB, kModeScan>(s, p, ct);
 }

@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(256) search_all(const float* code, int* mode_o
                                    : (static_cast<uint32_t>(i - npos) | 0x80000000u);
     const float xn = __uint_as_float(bits);
     uint32_t got;
-    if (mode == bq::kModeLut) got = bq::search<E, bq::kModeLut>(xn, s.tab, s.lut);
+    if (mode == bq::kModeLutF) got = bq::search<E, bq::kModeLutF>(xn, s.tab, s.lut);
+    else if (mode == bq::kModeLut) got = bq::search<E, bq::kModeLut>(xn, s.tab, s.lut);
     else if (mode == bq::kModeBsearch) got = bq::search<E, bq::kModeBsearch>(xn, s.tab, s.lut);
     else got = bq::search<E, bq::kModeScan>(xn, s.tab, s.lut);
     const uint32_t want = plain_scan<E>(xn, s.c);

@@ -362,7 +362,9 @@ def test_division_fp32_random(probes):
     assert mm.value == 0, f"{mm.value} quotients differ, first x={fa.value:#x} A={fb.value:#x}"
 
 
-@pytest.mark.parametrize("name,expect_mode", [("nf4", 0), ("fp4", 0), ("dyn8", 0)])
+# search forms: 0 = bucket table, integer select; 3 = bucket table, float
+# select (codes step by one at every threshold); FP4's +-0 pair makes one step 2
+@pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 0), ("dyn8", 3)])
 @pytest.mark.parametrize("force", [-1, 1], ids=["chosen", "bisection"])
 def test_search_exhaustive(probes, name, expect_mode, force):
     table = TABLES[name]
