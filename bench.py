@@ -19,7 +19,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -77,55 +76,58 @@ def step_bytes(n, nblk, only="all"):
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle reasons sampled with NVML every ~2 ms from a
+    thread while the timed region runs (the region is milliseconds long, far
+    shorter than nvidia-smi's sampling interval)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device):
-        self.lines = []
-        self.proc = None
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
         try:
+            import pynvml
+            pynvml.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except Exception:  # pragma: no cover - nvidia-smi missing
-            self.proc = None
+            self._nvml = pynvml
+            self._bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                          "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                          "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                          "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # pragma: no cover - no NVML
+            self.error = str(e)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv, h = self._nvml, self._h
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((mhz, reasons))
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
+                return
+            time.sleep(0.002)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            f = [v.strip() for v in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
+        self._stop.set()
+        if self.error and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml: {self.error}"]}
+        self._thread.join(timeout=1)
+        mhz = [m for m, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            for name, bit in self._bits.items():
+                if r & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
 
 
 # ------------------------------------------------------------------ peaks --
@@ -334,7 +336,7 @@ def run_ours(args, rank, world, local):
     barrier(world)
     torch.cuda.synchronize()
     sampler = ClockSampler(dev)
-    time.sleep(0.3)
+    time.sleep(0.01)
     for s in range(args.steps):
         ev[s][0].record(stream)
         for i, k in enumerate(names):

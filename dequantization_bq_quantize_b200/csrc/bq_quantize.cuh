@@ -107,6 +107,13 @@ __device__ __forceinline__ uint32_t bfi(uint32_t field, uint32_t base, int pos, 
 // it is only ever fed addresses computed from tile data loaded after the
 // mbarrier wait (itself after the table build and its barrier): the data
 // dependence keeps it after both.
+template <uint32_t OFF = 0>
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
 __device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
   uint2 v;
   asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -161,6 +168,13 @@ __device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut) {
   else return smem_u32(lut.e) + 8u * 1537u;
 }
 
+// Base of the split arrays of 16-entry tables (0 otherwise, unused).
+template <int E>
+__device__ __forceinline__ uint32_t lut_base_split(const Lut<E>& lut) {
+  if constexpr (E == 16) return smem_u32(lut.a) - 4u * (0x4B400000u - 15u);
+  else return 0u;
+}
+
 // Weight of element j within its 16-bit half of the output: a half holds 4
 // codes of 4 bits (element order in a byte: high nibble first) or 2 codes of
 // 8 bits, little-endian.
@@ -185,7 +199,8 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 //             bytes are merged with one byte permute per word.
 template <int DT, int E, int MODE>
 __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
-                                            uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
+                                            uint32_t t_base, uint32_t a_base,
+                                            uint32_t (&ow)[QOut<DT, E>::NW]) {
   using O = QOut<DT, E>;
   constexpr int NH = 2 * O::NW;                 // 16-bit halves
   constexpr int PER_HALF = O::EPT / NH;         // elements per half (4 or 2)
@@ -200,7 +215,15 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
     if constexpr (E == 16)
       unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
     const uint2 e0 = lds_u64(lut_addr<E>(b0, t_base));
-    const uint2 e1 = lds_u64(lut_addr<E>(b1, t_base));
+    uint2 e1;
+    if constexpr (E == 16) {
+      // second element from the split 32-bit arrays (lut.b is 128 bytes past
+      // lut.a): a_base = &lut.a[0] - 4 * (0x4B400000 - 15)
+      const uint32_t ad1 = __float_as_uint(b1) * 4u + a_base;
+      e1 = make_uint2(lds_u32<0>(ad1), lds_u32<128>(ad1));
+    } else {
+      e1 = lds_u64(lut_addr<E>(b1, t_base));
+    }
     const int j0 = 2 * i, j1 = 2 * i + 1;
     if constexpr (MODE == kModeLutF) {
       const float h0 = fma_sat(q0, kSelScale, __uint_as_float(e0.x));
@@ -251,7 +274,7 @@ __device__ __forceinline__ void encode_safe(const uint32_t (&w)[kThreadWords], c
 template <int DT, int E, int TPB, int MODE>
 __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uint32_t tile,
                                               int st, uint32_t par, uint32_t iter, int ct,
-                                              uint32_t t_base) {
+                                              uint32_t t_base, uint32_t a_base) {
   using O = QOut<DT, E>;
   constexpr int TE = kTileBytes / ElemBytes<DT>::value;
   constexpr int BPT = kQConsumers / TPB;
@@ -321,7 +344,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   // per-element condition is not needed, see div_fast); NaN fails both tests
   constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
-  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, ow);
+  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, a_base, ow);
   else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
@@ -368,12 +391,13 @@ template <int DT, int E, int TPB, int MODE>
 __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int ct) {
   constexpr int BPT = kQConsumers / TPB;
   const uint32_t t_base = lut_base<E>(s.lut);
+  const uint32_t a_base = lut_base_split<E>(s.lut);
   const uint32_t ntiles = static_cast<uint32_t>(p.full_tiles);  // < 2^24 (host check)
   uint32_t iter = 0;
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
     const int st = static_cast<int>(iter % kStages);
     const uint32_t par = (iter / kStages) & 1u;
-    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base)) break;
+    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base, a_base)) break;
   }
   // what the tiles did not cover: one quantization block per warp
   const int lane = ct & 31, cw = ct >> 5;
