@@ -246,7 +246,7 @@ def cpu_baseline(n, nblk, x_cpu):
     """Oracle timed on the host cores on a bounded sample (~10-30 s of CPU work)."""
     import oracle
     threads = oracle.host_threads()
-    n_s = min(n, 1 << 26)
+    n_s = min(n, 1 << 28)
     nblk_s = min(nblk, 1 << 18)
     xb = synth.to_numpy_bits(x_cpu[:n_s])
     nf4 = codebooks.nf4()
@@ -260,7 +260,7 @@ def cpu_baseline(n, nblk, x_cpu):
     dt = time.perf_counter() - t0
     byts = sum(step_bytes(n_s, nblk_s).values())
     return {"value": round(byts / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": (f"quantize+dequantize of the first 2^26 elements of the step's bf16 input "
+            "sample": (f"quantize+dequantize of the first 2^28 elements of the step's bf16 input "
                        f"({threads} threads over disjoint block ranges) and single-threaded "
                        f"Q8_0/Q4_0 dequant of 2^18 blocks each; {dt:.2f} s wall")}
 
