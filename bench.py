@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bq_inputs import codebooks, synth  # noqa: E402
+from dequantization_bq_quantize_b200 import shard  # noqa: E402
 
 METRIC = "quantize/dequantize HBM GB/s (in+out bytes) and % of B200 HBM peak"
 N_LARGE = synth.LARGE_N
@@ -50,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
+    ap.add_argument("--workload", choices=["step", "sweep", "llama"], default="step",
+                    help="step: the benchmark line; sweep / llama: informational tables")
     return ap.parse_args()
 
 
@@ -350,7 +353,7 @@ def run_ours(args, rank, world, local):
                   for i, k in enumerate(names)}
     max_ms = max_over_ranks(total_ms, world)
     ms_per_step = max_ms / args.steps
-    value = step_total * world / (ms_per_step / 1e3) / 1e9
+    value = shard.aggregate_gbs(step_total, world, ms_per_step)
 
     # ---- end to end: host buffers in, results back to the host, every step
     e2e = None
@@ -397,44 +400,230 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, w, names, stream, sh, byts, world):
-    """Same step through the public API with host buffers: pinned host->device
-    copy of the step's inputs and device->host copy of its results, inside the
-    timed region, every step."""
-    pin = lambda t: t.pin_memory()  # noqa: E731
-    xh = pin(w.x_cpu)
-    q8h, q4h = pin(w.q8_cpu), pin(w.q4_cpu)
-    outs = {"quantize": [w.absmax, w.q], "dequantize": [w.y], "q8_0": [w.y8], "q4_0": [w.y4]}
-    ins = {"quantize": [(w.x, xh)], "dequantize": [], "q8_0": [(w.q8, q8h)],
-           "q4_0": [(w.q4, q4h)]}
-    hosts = {k: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs[k]]
-             for k in names}
-    h2d = sum(h.numel() * h.element_size() for k in names for _, h in ins[k])
-    d2h = sum(t.numel() * t.element_size() for k in names for t in outs[k])
-    steps = max(1, min(args.steps, 5))
+def run_e2e(args, w, names, stream, sh, byts, world, chunks=8):
+    """Same step through the public API with host buffers, every step: pinned
+    host->device copy of the step's inputs and device->host copy of all its
+    results inside the timed region.  The work is cut into `chunks` pieces on
+    quantization-block boundaries (blocks are independent, so the results are
+    identical) and pipelined over three streams: copies in, kernels, copies
+    out, so that PCIe traffic in both directions overlaps the kernels."""
+    bq = w.bq
+    n, nblk = w.n, w.nblk
+    xh = w.x_cpu.pin_memory()
+    q8h, q4h = w.q8_cpu.pin_memory(), w.q4_cpu.pin_memory()
+    pinned = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
+    ah, qh, yh, y8h, y4h = pinned(w.absmax), pinned(w.q), pinned(w.y), pinned(w.y8), pinned(w.y4)
+    s_in, s_k, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    # chunk boundaries: whole blocks (and an even element count) per chunk
+    per = -(-w.nb // chunks) * BS
+    ranges = [(lo, min(n, lo + per)) for lo in range(0, n, per)]
+    gper = -(-nblk // chunks)
+    granges = [(lo, min(nblk, lo + gper)) for lo in range(0, nblk, gper)]
+    h2d = d2h = 0
+
+    # per chunk: the previous step's kernel and copy-out events (buffer reuse)
+    prev_k = [None] * len(ranges)
+    prev_out = [None] * len(ranges)
 
     def one():
-        for k in names:
-            for d, h in ins[k]:
-                d.copy_(h, non_blocking=True)
-            w.launch(k, sh)
-            for d, h in zip(outs[k], hosts[k]):
-                h.copy_(d, non_blocking=True)
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        for ci in range(len(ranges)):
+            lo, hi = ranges[ci]
+            glo, ghi = granges[ci] if ci < len(granges) else (0, 0)
+            b0, b1 = lo // BS, -(-hi // BS)
+            e_in = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                if prev_k[ci] is not None:
+                    s_in.wait_event(prev_k[ci])  # inputs still read by last step's kernels
+                if "quantize" in names:
+                    w.x[lo:hi].copy_(xh[lo:hi], non_blocking=True)
+                    h2d += (hi - lo) * 2
+                if "q8_0" in names and ghi > glo:
+                    w.q8[glo * 34:ghi * 34].copy_(q8h[glo * 34:ghi * 34], non_blocking=True)
+                    h2d += (ghi - glo) * 34
+                if "q4_0" in names and ghi > glo:
+                    w.q4[glo * 18:ghi * 18].copy_(q4h[glo * 18:ghi * 18], non_blocking=True)
+                    h2d += (ghi - glo) * 18
+                e_in.record(s_in)
+            e_k = torch.cuda.Event()
+            with torch.cuda.stream(s_k):
+                s_k.wait_event(e_in)
+                if prev_out[ci] is not None:
+                    s_k.wait_event(prev_out[ci])  # outputs still copied out by last step
+                ks = s_k.cuda_stream
+                if "quantize" in names:
+                    st = bq.bq_quantize_blockwise(w.x.data_ptr() + 2 * lo, bq.BQ_BF16, hi - lo, BS,
+                                                  w.code.data_ptr(), 16,
+                                                  w.absmax.data_ptr() + 4 * b0,
+                                                  w.q.data_ptr() + lo // 2, ks)
+                    assert st == bq.BQ_OK, bq.bq_last_cuda_error()
+                if "dequantize" in names:
+                    st = bq.bq_dequantize_blockwise(w.q.data_ptr() + lo // 2,
+                                                    w.absmax.data_ptr() + 4 * b0, hi - lo, BS,
+                                                    w.code.data_ptr(), 16,
+                                                    w.y.data_ptr() + 2 * lo, bq.BQ_BF16, ks)
+                    assert st == bq.BQ_OK, bq.bq_last_cuda_error()
+                if "q8_0" in names and ghi > glo:
+                    st = bq.bq_dequant_q8_0(w.q8.data_ptr() + 34 * glo, ghi - glo,
+                                            w.y8.data_ptr() + 64 * glo, bq.BQ_BF16, ks)
+                    assert st == bq.BQ_OK, bq.bq_last_cuda_error()
+                if "q4_0" in names and ghi > glo:
+                    st = bq.bq_dequant_q4_0(w.q4.data_ptr() + 18 * glo, ghi - glo,
+                                            w.y4.data_ptr() + 64 * glo, bq.BQ_BF16, ks)
+                    assert st == bq.BQ_OK, bq.bq_last_cuda_error()
+                e_k.record(s_k)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e_k)
+                if "quantize" in names:
+                    ah[b0:b1].copy_(w.absmax[b0:b1], non_blocking=True)
+                    qh[lo // 2:(hi + 1) // 2].copy_(w.q[lo // 2:(hi + 1) // 2], non_blocking=True)
+                    d2h += (b1 - b0) * 4 + ((hi + 1) // 2 - lo // 2)
+                if "dequantize" in names:
+                    yh[lo:hi].copy_(w.y[lo:hi], non_blocking=True)
+                    d2h += (hi - lo) * 2
+                if "q8_0" in names and ghi > glo:
+                    y8h[32 * glo:32 * ghi].copy_(w.y8[32 * glo:32 * ghi], non_blocking=True)
+                    d2h += (ghi - glo) * 64
+                if "q4_0" in names and ghi > glo:
+                    y4h[32 * glo:32 * ghi].copy_(w.y4[32 * glo:32 * ghi], non_blocking=True)
+                    d2h += (ghi - glo) * 64
+                e_out = torch.cuda.Event()
+                e_out.record(s_out)
+            prev_k[ci], prev_out[ci] = e_k, e_out
 
     one()
     torch.cuda.synchronize()
     barrier(world)
+    steps = max(1, min(args.steps, 5))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(s_in)
     for _ in range(steps):
         one()
-    e1.record(stream)
+    for st_ in (s_in, s_k):
+        ev = torch.cuda.Event()
+        ev.record(st_)
+        s_out.wait_event(ev)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    # the pipelined, chunked calls must give the device-resident results
+    for host, dev in ((ah, w.absmax), (qh, w.q), (yh, w.y), (y8h, w.y8), (y4h, w.y4)):
+        k = min(dev.numel(), 1 << 20)
+        if not (torch.equal(host[:k], dev[:k].cpu()) and torch.equal(host[-k:], dev[-k:].cpu())):
+            raise RuntimeError("end-to-end results differ from the device-resident run")
     total = sum(byts.values()) * world
     return {"value": round(total / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
-            "steps": steps}
+            "steps": steps, "pipeline": f"{len(ranges)} chunks over 3 streams (in / kernels / out)"}
+
+
+# ------------------------------------------------------ informational ---
+
+def _timed(fn, reps, flush=None):
+    """Device time (ms) of one fn() call.  With `flush`, every call is
+    preceded by a write of the flush buffer (larger than L2): `reps` pairs
+    (flush, fn) are queued back to back and the time of `reps` flushes alone
+    is subtracted, so neither host launch latency nor the flush is counted."""
+    def batch(with_fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            if flush is not None:
+                flush.zero_()
+            if with_fn:
+                fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+    batch(True)  # warm
+    if flush is None:
+        return batch(True) / reps
+    return max(0.0, (batch(True) - batch(False)) / reps)
+
+
+def run_sweep(args):
+    """45 cells: {fp16, bf16, fp32} x {NF4, FP4, dyn8} x bs {32, 64, 256, 1024,
+    4096} at n = 8388608 + 37 with one all-zero block; quantize and dequantize
+    (to the input dtype) timed separately with a 512 MiB L2 flush before each
+    repetition (the tensors fit in L2)."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(1 << 29, dtype=torch.uint8, device=dev)
+    cells = []
+    ci = 0
+    for dtype in ("f16", "bf16", "f32"):
+        for name in ("nf4", "fp4", "dyn8"):
+            code = torch.from_numpy(codebooks.get(name)).to(dev)
+            for bs in (32, 64, 256, 1024, 4096):
+                x = synth.sweep(dtype, bs, seed=1 + ci).to(dev)
+                n = x.numel()
+                a, q = bq.quantize_blockwise(x, code, bs)
+                y = bq.dequantize_blockwise(q, a, n, bs, code, dtype=x.dtype)
+                eb = x.element_size()
+                nbytes = n * eb + q.numel() + 4 * a.numel()
+                tq = _timed(lambda: bq.quantize_blockwise(x, code, bs, absmax=a, out=q), 20, flush)
+                td = _timed(lambda: bq.dequantize_blockwise(q, a, n, bs, code, out=y), 20, flush)
+                cells.append({"dtype": dtype, "codebook": name, "blocksize": bs,
+                              "quantize_us": round(tq * 1e3, 1),
+                              "quantize_gbs": round(nbytes / (tq / 1e3) / 1e9, 1),
+                              "dequantize_us": round(td * 1e3, 1),
+                              "dequantize_gbs": round(nbytes / (td / 1e3) / 1e9, 1)})
+                ci += 1
+    print(json.dumps({"workload": "sweep", "n": synth.SWEEP_N, "cells": cells}), flush=True)
+
+
+def run_llama(args):
+    """The 224 weight matrices of a Llama-3-8B-shaped model (32 layers),
+    bf16 N(0, 0.02) drawn on the device from a seeded generator per matrix;
+    quantize then dequantize of every matrix back-to-back on one stream."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    code = torch.from_numpy(codebooks.nf4()).to(dev)
+    mats, outs = [], []
+    total = 0
+    for layer, i, name, r, c, seed in synth.llama_matrices():
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        x = torch.randn(r * c, generator=g, device=dev, dtype=torch.float32).mul_(0.02).to(
+            torch.bfloat16)
+        n = x.numel()
+        a = torch.empty((n + BS - 1) // BS, dtype=torch.float32, device=dev)
+        q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        y = torch.empty_like(x)
+        mats.append(x)
+        outs.append((a, q, y))
+        total += 2 * quant_bytes(n, BS)
+
+    def everything():
+        for x, (a, q, y) in zip(mats, outs):
+            bq.quantize_blockwise(x, code, BS, absmax=a, out=q)
+            bq.dequantize_blockwise(q, a, x.numel(), BS, code, out=y)
+
+    for _ in range(max(1, args.warmup)):
+        everything()
+    torch.cuda.synchronize()
+    ms_eager = _timed(everything, max(1, args.steps))
+    # the 448 launches captured once in a CUDA graph (the calls allocate
+    # nothing and never synchronise), replayed: device time without host
+    # launch overhead
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            everything()
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    ms = _timed(graph.replay, max(1, args.steps))
+    print(json.dumps({"workload": "llama3-8b-shaped weight set", "matrices": len(mats),
+                      "eager_ms": round(ms_eager, 3),
+                      "elements": sum(m.numel() for m in mats), "bytes": total,
+                      "ms": round(ms, 3), "gbs": round(total / (ms / 1e3) / 1e9, 1),
+                      "frac_of_measured_peak": round(total / (ms / 1e3) / 1e9 / measured_peaks()[0], 4)}),
+          flush=True)
 
 
 def main():
@@ -443,6 +632,10 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "sweep":
+            run_sweep(args)
+        elif args.workload == "llama":
+            run_llama(args)
         else:
             run_ours(args, rank, world, local)
     finally:

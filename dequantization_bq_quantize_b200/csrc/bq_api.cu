@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "bq_dequant.cuh"
 #include "bq_gguf.cuh"
@@ -98,6 +99,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
   return fn;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel on the stream finishes; every kernel waits for it
+// (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool valid_dtype(int d) { return d == BQ_F32 || d == BQ_F16 || d == BQ_BF16; }
 int elem_bytes(int d) { return d == BQ_F32 ? 4 : 2; }
 bool valid_blocksize(int32_t bs) { return bs >= 32 && bs <= 4096 && (bs & (bs - 1)) == 0; }
@@ -123,8 +143,7 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
   if (want < 1) want = 1;
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  kernel<<<grid, bq::kQThreads, smem, stream>>>(map, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kernel, grid, bq::kQThreads, smem, stream, map, p);
   return e == cudaSuccess ? BQ_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -170,8 +189,7 @@ bq_status launch_dequant(const bq::DParams& p, int dev, int sms, cudaStream_t st
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
-  kernel<<<static_cast<int>(want), bq::kDThreads, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kDThreads, 0, stream, p);
   return e == cudaSuccess ? BQ_OK : cuda_fail(e, "dequantize launch");
 }
 
@@ -195,8 +213,7 @@ bq_status launch_gguf(const bq::GParams& p, int dev, int sms, cudaStream_t strea
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
-  kernel<<<static_cast<int>(want), bq::kGThreads, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kGThreads, 0, stream, p);
   return e == cudaSuccess ? BQ_OK : cuda_fail(e, "gguf dequant launch");
 }
 

@@ -179,4 +179,13 @@ __device__ __forceinline__ void named_sync(int id, int count) {
 
 __device__ __forceinline__ void record_fault(uint32_t bit) { atomicOr(&g_fault, bit); }
 
+// Programmatic dependent launch.  Kernels are launched so that they may start
+// while the previous kernel on the stream is finishing; each one waits for
+// that kernel's completion (and its memory) before touching global memory, and
+// lets its own dependents start launching right away.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace bq

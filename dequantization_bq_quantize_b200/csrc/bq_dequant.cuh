@@ -10,7 +10,9 @@
 // store is 512 contiguous bytes and every warp-wide code load is contiguous
 // too.  A chunk never straddles a quantization block (blocksize >= 32), so it
 // needs one absmax.  Each thread handles eight chunks a grid-stride apart per
-// iteration with all loads issued first.
+// iteration with all loads issued first.  (Issuing the next iteration's loads
+// before decoding these was tried and measured slower: the extra registers
+// cost more occupancy than the overlap won.)
 // 4-bit codes: a byte holds the codes of two neighbouring elements, so the
 // shared table is indexed by the whole byte and holds the pair
 // (code[byte >> 4], code[byte & 15]): one 64-bit shared load and one packed
@@ -105,6 +107,8 @@ __device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, uint32_t t_base)
 template <int E, int OT>
 __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
   __shared__ DSmem<E> s;
+  pdl_release();
+  pdl_wait();  // codes, absmax, codebook and y may belong to the previous kernel
   for (int i = threadIdx.x; i < E; i += blockDim.x) s.code[i] = p.code[i];
   __syncthreads();
   if constexpr (E == 16) {

@@ -14,7 +14,7 @@
 // 1088 B for Q8_0, 576 B for Q4_0).  A group of 8 blocks is 272 or 144 bytes,
 // a whole number of 16-byte chunks, so in a 16-byte aligned stream every group
 // starts aligned and the warp stages its 4 groups into its shared buffer with
-// up to three 16-byte loads per lane, all issued before any is used.  Lane l
+// up to three 16-byte loads per lane, fetched into registers one step ahead.  Lane l
 // then decodes 8 outputs of block l/4 of each group and writes them as one
 // 16-byte store, so each warp store covers 512 contiguous bytes of bf16
 // output.  Bytes become floats with the 2^23 trick: a byte b placed in the low
@@ -128,25 +128,37 @@ __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
   uint8_t* wb = buf[warp];
   const int64_t nsteps = (p.n_blocks + STEP_BLOCKS - 1) / STEP_BLOCKS;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kGThreads / 32);
+  pdl_release();
+  pdl_wait();  // blocks and y may belong to the previous kernel
 
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (kGThreads / 32) + warp; g < nsteps;
-       g += nwarps) {
+  // 16-byte chunks of a whole step, prefetched into registers one step ahead
+  auto full_step = [&](int64_t g) {
+    return p.vec && g < nsteps && (g + 1) * STEP_BLOCKS <= p.n_blocks;
+  };
+  auto fetch = [&](int64_t g, uint4 (&v)[LOADS]) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.blocks + g * STEP_BLOCKS * BB);
+#pragma unroll
+    for (int i = 0; i < LOADS; ++i) {
+      const int c = lane + 32 * i;
+      if (c < STEP_CHUNKS) v[i] = __ldg(src + c);
+    }
+  };
+  uint4 vn[LOADS];
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (kGThreads / 32) + warp;
+  if (full_step(g)) fetch(g, vn);
+
+  for (; g < nsteps; g += nwarps) {
     const int64_t blk0 = g * STEP_BLOCKS;
     const int nblk = static_cast<int>(min(static_cast<int64_t>(STEP_BLOCKS), p.n_blocks - blk0));
-    const uint8_t* src = p.blocks + blk0 * BB;
-    if (p.vec && nblk == STEP_BLOCKS) {
-      uint4 v[LOADS];
+    if (full_step(g)) {
 #pragma unroll
       for (int i = 0; i < LOADS; ++i) {
         const int c = lane + 32 * i;
-        if (c < STEP_CHUNKS) v[i] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+        if (c < STEP_CHUNKS) reinterpret_cast<uint4*>(wb)[c] = vn[i];
       }
-#pragma unroll
-      for (int i = 0; i < LOADS; ++i) {
-        const int c = lane + 32 * i;
-        if (c < STEP_CHUNKS) reinterpret_cast<uint4*>(wb)[c] = v[i];
-      }
+      if (full_step(g + nwarps)) fetch(g + nwarps, vn);
     } else {
+      const uint8_t* src = p.blocks + blk0 * BB;
       for (int i = lane; i < nblk * BB; i += 32) wb[i] = src[i];
     }
     __syncwarp();

@@ -424,6 +424,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
     s.cabort[1] = 0;
     fence_mbar_init();
   }
+  pdl_release();
+  pdl_wait();  // inputs, codebook and outputs may belong to the previous kernel
   __syncthreads();
 
   if (warp == 0) {
