@@ -84,19 +84,42 @@ def large_outliers(n=LARGE_N, seed=3, std=0.02, outlier_std=0.4, rate=0.001,
     return out, count
 
 
+# GGUF block types: bytes per block and the byte offsets of the fp16 fields
+# (scale d, min m, super-block dmin) as (offset, signed).  Format facts only.
+GGUF_LAYOUT = {
+    "q8_0": (34, ((0, False),)),
+    "q4_0": (18, ((0, False),)),
+    "q4_1": (20, ((0, False), (2, True))),
+    "q5_0": (22, ((0, False),)),
+    "q5_1": (24, ((0, False), (2, True))),
+    "q4_k": (144, ((0, False), (2, False))),
+    "q6_k": (210, ((208, False),)),
+}
+
+
 def gguf_blocks(n_blocks, kind, seed=4):
-    """GGUF Q8_0 (34 B) or Q4_0 (18 B) blocks as a uint8 numpy array
-    [n_blocks, block_bytes]: fp16 d little-endian in bytes 0..1, then the
-    quant bytes drawn uniformly from 0..255."""
-    qbytes = {"q8_0": 32, "q4_0": 16}[kind]
+    """GGUF blocks of `kind` as a uint8 numpy array [n_blocks, block_bytes].
+
+    Each fp16 field is |N(0,1)| * 0.01 (a signed N(0,1) * 0.01 for a min
+    field), stored little-endian at its offset; every other byte (quant bytes,
+    high-bit words, packed sub-block scales) is uniform on 0..255."""
+    bb, fields = GGUF_LAYOUT[kind]
     g = _gen(seed)
-    d = torch.randn(n_blocks, generator=g, dtype=torch.float32).abs_().mul_(0.01)
-    d16 = d.to(torch.float16).numpy().view(np.uint16)
-    qs = torch.randint(0, 256, (n_blocks, qbytes), generator=g, dtype=torch.uint8).numpy()
-    blocks = np.empty((n_blocks, 2 + qbytes), np.uint8)
-    blocks[:, 0] = (d16 & 0xFF).astype(np.uint8)
-    blocks[:, 1] = (d16 >> 8).astype(np.uint8)
-    blocks[:, 2:] = qs
+    vals = []
+    for _, signed in fields:
+        d = torch.randn(n_blocks, generator=g, dtype=torch.float32)
+        if not signed:
+            d.abs_()
+        vals.append(d.mul_(0.01).to(torch.float16).numpy().view(np.uint16))
+    rest = bb - 2 * len(fields)
+    qs = torch.randint(0, 256, (n_blocks, rest), generator=g, dtype=torch.uint8).numpy()
+    blocks = np.empty((n_blocks, bb), np.uint8)
+    free = np.ones(bb, bool)
+    for (off, _), h in zip(fields, vals):
+        blocks[:, off] = (h & 0xFF).astype(np.uint8)
+        blocks[:, off + 1] = (h >> 8).astype(np.uint8)
+        free[off:off + 2] = False
+    blocks[:, free] = qs
     return blocks
 
 

@@ -1,4 +1,4 @@
-"""CPU oracle for blockwise codebook quantization and GGUF Q8_0/Q4_0 dequantization.
+"""CPU oracle for blockwise codebook quantization and GGUF block dequantization.
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
@@ -19,6 +19,10 @@ import numpy as np
 from . import build as _build
 
 DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
+
+# GGUF block types: (elements per block, bytes per block)
+GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32, 22),
+              "q5_1": (32, 24), "q4_k": (256, 144), "q6_k": (256, 210)}
 _ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
 
 _lib = None
@@ -53,6 +57,10 @@ def _declare(L):
     L.bqo_dequant_q8_0.restype = c_int
     L.bqo_dequant_q4_0.argtypes = [c_void_p, c_int64, c_void_p, c_int]
     L.bqo_dequant_q4_0.restype = c_int
+    for kind in GGUF_TYPES:
+        f = getattr(L, "bqo_dequant_" + kind)
+        f.argtypes = [c_void_p, c_int64, c_void_p, c_int]
+        f.restype = c_int
     return L
 
 
@@ -133,6 +141,18 @@ def dequant_q4_0(blocks, ydtype, L=None):
     nblk = blocks.size // 18
     y = _out_array(32 * nblk, ydtype)
     if L.bqo_dequant_q4_0(_ptr(blocks), nblk, _ptr(y), DTYPES[ydtype]) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return y
+
+
+def dequant_gguf(kind, blocks, ydtype, L=None):
+    """Dequantize GGUF blocks of type `kind` (a key of GGUF_TYPES)."""
+    L = L or lib()
+    per, bb = GGUF_TYPES[kind]
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8).reshape(-1)
+    nblk = blocks.size // bb
+    y = _out_array(per * nblk, ydtype)
+    if getattr(L, "bqo_dequant_" + kind)(_ptr(blocks), nblk, _ptr(y), DTYPES[ydtype]) != 0:
         raise ValueError("oracle rejected the arguments")
     return y
 

@@ -224,3 +224,133 @@ int bqo_dequant_q4_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
     }
     return 0;
 }
+
+/* ------------------------------------------------------- more GGUF types -- */
+
+static float half_at(const uint8_t *p) { return bqo_f16_to_f32((uint16_t)(p[0] | (p[1] << 8))); }
+
+static uint32_t u32_at(const uint8_t *p)
+{
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+
+int bqo_dequant_q4_1(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 20 * k;
+        float d = half_at(blk), m = half_at(blk + 2);
+        for (int j = 0; j < 16; ++j) {
+            int lo = blk[4 + j] & 15, hi = blk[4 + j] >> 4;
+            store_elem(y, ydtype, 32 * k + j, d * (float)lo + m);
+            store_elem(y, ydtype, 32 * k + 16 + j, d * (float)hi + m);
+        }
+    }
+    return 0;
+}
+
+/* 5-bit value of element e (0..31) of a Q5 block: nibble plus bit e of qh */
+static int q5_value(const uint8_t *qs, uint32_t qh, int e)
+{
+    int nib = e < 16 ? (qs[e] & 15) : (qs[e - 16] >> 4);
+    return nib | (int)(((qh >> e) & 1u) << 4);
+}
+
+int bqo_dequant_q5_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 22 * k;
+        float d = half_at(blk);
+        uint32_t qh = u32_at(blk + 2);
+        for (int e = 0; e < 32; ++e)
+            store_elem(y, ydtype, 32 * k + e, d * (float)(q5_value(blk + 6, qh, e) - 16));
+    }
+    return 0;
+}
+
+int bqo_dequant_q5_1(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 24 * k;
+        float d = half_at(blk), m = half_at(blk + 2);
+        uint32_t qh = u32_at(blk + 4);
+        for (int e = 0; e < 32; ++e)
+            store_elem(y, ydtype, 32 * k + e, d * (float)q5_value(blk + 8, qh, e) + m);
+    }
+    return 0;
+}
+
+/* Q4_K: the 6-bit scale and min of sub-block i from the 12 packed bytes:
+ * sub-blocks 0..3 keep theirs in the low 6 bits of bytes i and i + 4;
+ * sub-blocks 4..7 take their low 4 bits from byte i + 4 (scale: low nibble,
+ * min: high nibble) and their top 2 bits from the top 2 bits of bytes i - 4
+ * (scale) and i (min). */
+static void q4k_scale_min(const uint8_t *sc, int i, int *scale, int *mn)
+{
+    if (i < 4) {
+        *scale = sc[i] & 63;
+        *mn = sc[i + 4] & 63;
+    } else {
+        *scale = (sc[i + 4] & 15) | ((sc[i - 4] >> 6) << 4);
+        *mn = (sc[i + 4] >> 4) | ((sc[i] >> 6) << 4);
+    }
+}
+
+int bqo_dequant_q4_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 144 * k;
+        float d = half_at(blk), dmin = half_at(blk + 2);
+        const uint8_t *scales = blk + 4, *qs = blk + 16;
+        /* 4 groups of 64 elements: 32 bytes of qs each; low nibbles form
+         * sub-block 2g, high nibbles sub-block 2g + 1 */
+        for (int g = 0; g < 4; ++g) {
+            for (int h = 0; h < 2; ++h) {
+                int sci, mni;
+                q4k_scale_min(scales, 2 * g + h, &sci, &mni);
+                float a = d * (float)sci, b = dmin * (float)mni;
+                for (int l = 0; l < 32; ++l) {
+                    int q = h ? (qs[32 * g + l] >> 4) : (qs[32 * g + l] & 15);
+                    store_elem(y, ydtype, 256 * k + 64 * g + 32 * h + l, a * (float)q - b);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 210 * k;
+        const uint8_t *ql = blk, *qh = blk + 128;
+        const int8_t *sc = (const int8_t *)(blk + 192);
+        float d = half_at(blk + 208);
+        /* two halves of 128; in a half, element 32 * c + l (c = 0..3, l < 32)
+         * takes its low 4 bits from ql[l + 32 * (c & 1)] (low nibble for c < 2,
+         * high nibble otherwise), its top 2 bits from bits 2c, 2c+1 of qh[l],
+         * and scale sc[l / 16 + 2 * c] */
+        for (int n = 0; n < 2; ++n) {
+            for (int c = 0; c < 4; ++c) {
+                for (int l = 0; l < 32; ++l) {
+                    int lo4 = ql[64 * n + l + 32 * (c & 1)];
+                    lo4 = c < 2 ? (lo4 & 15) : (lo4 >> 4);
+                    int hi2 = (qh[32 * n + l] >> (2 * c)) & 3;
+                    int q = (lo4 | (hi2 << 4)) - 32;
+                    float a = d * (float)sc[8 * n + l / 16 + 2 * c];
+                    store_elem(y, ydtype, 256 * k + 128 * n + 32 * c + l, a * (float)q);
+                }
+            }
+        }
+    }
+    return 0;
+}

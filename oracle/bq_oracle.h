@@ -1,6 +1,7 @@
 /*
  * bq_oracle.h - plain, slow, single-threaded CPU reference for blockwise
- * codebook quantization / dequantization and GGUF Q8_0 / Q4_0 dequantization.
+ * codebook quantization / dequantization and GGUF block dequantization
+ * (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the library path may include, link
  * or call this code: only the tests, the package's smoke check and the
@@ -15,6 +16,11 @@
  *  - "ComfyUI-GGUF PR #472, Cache device-side constants in dequant kernels",
  *    Problem section (Q4_0 low nibble then high nibble, shift vector [0, 4])
  *    and the Verification table (Q8_0 and Q4_0 rows).
+ *  - The same page's Verification table also lists Q4_1, Q5_0, Q5_1, Q4_K
+ *    and Q6_K (4096 blocks, bf16 target, bit-identical).  The pages do not
+ *    spell out those block layouts; the functions below follow the GGUF
+ *    format's published block layouts, and the tests pin them against the
+ *    gguf package's own dequantizer and hand-worked blocks.
  *  - "Model-Optimizer PR #2448" review notes: lowest index wins on equal
  *    error; fused multiply-add changes near-ties, so this file is compiled
  *    with contraction off (-ffp-contract=off) and no fast-math.
@@ -66,6 +72,29 @@ int bqo_dequant_q8_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
 /* GGUF Q4_0: 18-byte blocks {fp16 d, uint8 qs[16]};
  * y[32k+j] = d*((qs[j] & 15) - 8), y[32k+16+j] = d*((qs[j] >> 4) - 8). */
 int bqo_dequant_q4_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q4_1: 20-byte blocks {fp16 d, fp16 m, uint8 qs[16]};
+ * y[32k+j] = d*(qs[j] & 15) + m, y[32k+16+j] = d*(qs[j] >> 4) + m. */
+int bqo_dequant_q4_1(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q5_0: 22-byte blocks {fp16 d, uint32 qh (little endian), uint8 qs[16]};
+ * element e's 5-bit value is its nibble (as Q4_0) plus bit e of qh as bit 4;
+ * y = d*(value - 16). */
+int bqo_dequant_q5_0(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q5_1: 24-byte blocks {fp16 d, fp16 m, uint32 qh, uint8 qs[16]};
+ * y = d*value + m. */
+int bqo_dequant_q5_1(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q4_K: 144-byte super-blocks of 256 {fp16 d, fp16 dmin, uint8 scales[12],
+ * uint8 qs[128]}: 8 sub-blocks of 32 with 6-bit scales sc[i] and mins mn[i];
+ * y = d*sc*q - dmin*mn with q the 4-bit value. */
+int bqo_dequant_q4_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q6_K: 210-byte super-blocks of 256 {uint8 ql[128], uint8 qh[64],
+ * int8 scales[16], fp16 d}: 16 sub-blocks of 16, y = d*scale*(q - 32) with q
+ * the 6-bit value (4 low bits from ql, 2 high bits from qh). */
+int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
 
 #ifdef __cplusplus
 }

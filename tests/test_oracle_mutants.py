@@ -39,6 +39,19 @@ MUTANTS = [
     ("q8_unsigned", "int qv = (int)(int8_t)blk[2 + j];", "int qv = (int)blk[2 + j];"),
     ("q4_nibbles_swapped", "int lo = blk[2 + j] & 15;", "int lo = blk[2 + j] >> 4;"),
     ("q4_no_offset", "d * (float)(lo - 8)", "d * (float)(lo)"),
+    ("q4_1_min_dropped", "d * (float)lo + m);", "d * (float)lo);"),
+    ("q5_qh_bit_order", "(((qh >> e) & 1u) << 4)", "(((qh >> (31 - e)) & 1u) << 4)"),
+    ("q5_0_offset", "(float)(q5_value(blk + 6, qh, e) - 16)", "(float)(q5_value(blk + 6, qh, e) - 15)"),
+    ("q5_1_qh_offset", "uint32_t qh = u32_at(blk + 4);", "uint32_t qh = u32_at(blk + 2);"),
+    ("q4k_scale_min_nibbles", "*scale = (sc[i + 4] & 15) | ((sc[i - 4] >> 6) << 4);",
+     "*scale = (sc[i + 4] >> 4) | ((sc[i - 4] >> 6) << 4);"),
+    ("q4k_top_bits_source", "*mn = (sc[i + 4] >> 4) | ((sc[i] >> 6) << 4);",
+     "*mn = (sc[i + 4] >> 4) | ((sc[i - 4] >> 6) << 4);"),
+    ("q4k_nibble_halves", "int q = h ? (qs[32 * g + l] >> 4) : (qs[32 * g + l] & 15);",
+     "int q = h ? (qs[32 * g + l] & 15) : (qs[32 * g + l] >> 4);"),
+    ("q6k_offset", "int q = (lo4 | (hi2 << 4)) - 32;", "int q = (lo4 | (hi2 << 4)) - 31;"),
+    ("q6k_scale_index", "sc[8 * n + l / 16 + 2 * c]", "sc[8 * n + l / 16 + c]"),
+    ("q6k_qh_shift", "int hi2 = (qh[32 * n + l] >> (2 * c)) & 3;", "int hi2 = (qh[32 * n + l] >> c) & 3;"),
     ("f16_bias", "ldexpf((float)(m + 1024), e - 25)", "ldexpf((float)(m + 1024), e - 24)"),
     ("bf16_ties_away", "if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))",
      "if (lower >= 0x8000u)"),

@@ -85,17 +85,22 @@ def _load_hand_blocks():
                 continue
             parts = line.split()
             blk = np.frombuffer(bytes.fromhex(parts[1]), np.uint8)
-            vals = np.array([float(v) for v in parts[2:]], np.float32)
-            recs.append((parts[0], blk, vals))
+            vals = []
+            for tok in parts[2:]:
+                v, _, k = tok.partition("*")
+                vals += [float(v)] * (int(k) if k else 1)
+            recs.append((parts[0], blk, np.array(vals, np.float32)))
     return recs
 
 
 def test_gguf_hand_worked_blocks():
     recs = _load_hand_blocks()
-    assert len(recs) == 7
+    assert len(recs) == 12
+    assert {r[0] for r in recs} == set(oracle.GGUF_TYPES)
     for kind, blk, expect in recs:
-        assert blk.size == (34 if kind == "q8_0" else 18)
-        fn = oracle.dequant_q8_0 if kind == "q8_0" else oracle.dequant_q4_0
+        per, bb = oracle.GGUF_TYPES[kind]
+        assert blk.size == bb and expect.size == per, kind
+        fn = lambda b, dt, kind=kind: oracle.dequant_gguf(kind, b, dt)
         y = fn(blk, "f32")
         # bit equality (keeps the sign of zero: d = -0.5 times q = 0 is -0)
         assert np.array_equal(y.view(np.uint32), expect.view(np.uint32)), (kind, y, expect)
@@ -135,15 +140,47 @@ def test_gguf_closed_form_exhaustive_bytes():
 
 
 def test_gguf_matches_gguf_package():
-    """Independent cross-check: the installed gguf package's numpy dequantizer."""
+    """Independent cross-check: the installed gguf package's numpy dequantizer,
+    every block type, bit for bit (including the sign of zero)."""
     gq = pytest.importorskip("gguf.quants")
     import gguf
-    for kind, qt in (("q8_0", gguf.GGMLQuantizationType.Q8_0),
-                     ("q4_0", gguf.GGMLQuantizationType.Q4_0)):
-        blocks = synth.gguf_blocks(512, kind, seed=11)
+    T = gguf.GGMLQuantizationType
+    qts = {"q8_0": T.Q8_0, "q4_0": T.Q4_0, "q4_1": T.Q4_1, "q5_0": T.Q5_0, "q5_1": T.Q5_1,
+           "q4_k": T.Q4_K, "q6_k": T.Q6_K}
+    assert set(qts) == set(oracle.GGUF_TYPES)
+    for kind, qt in qts.items():
+        blocks = synth.gguf_blocks(512 if oracle.GGUF_TYPES[kind][0] == 32 else 64, kind, seed=11)
         ref = gq.dequantize(blocks.reshape(-1), qt).astype(np.float32).reshape(-1)
-        fn = oracle.dequant_q8_0 if kind == "q8_0" else oracle.dequant_q4_0
-        assert np.array_equal(fn(blocks, "f32"), ref)
+        y = oracle.dequant_gguf(kind, blocks, "f32")
+        assert np.array_equal(y.view(np.uint32), ref.view(np.uint32)), kind
+        if kind == "q8_0":
+            assert np.array_equal(oracle.dequant_q8_0(blocks, "f32"), y)
+        if kind == "q4_0":
+            assert np.array_equal(oracle.dequant_q4_0(blocks, "f32"), y)
+
+
+def test_gguf_more_types_exact_products():
+    """Closed form of the scale arithmetic: every product in these formats is
+    exact in binary32 (fp16 d: 11 bits; Q4_K d*sc*q: 11+6+4 bits; Q6_K
+    d*sc*(q-32): 11+7+5 bits), so with exact rationals the only rounding is
+    the add of a min, and for Q5_0 / Q6_K there is none at all."""
+    for kind in ("q5_0", "q6_k"):
+        blocks = synth.gguf_blocks(64, kind, seed=21)
+        y = oracle.dequant_gguf(kind, blocks, "f32")
+        # dequantizing in double gives bit-identical values: no rounding occurred
+        per, bb = oracle.GGUF_TYPES[kind]
+        d_off = 0 if kind == "q5_0" else 208
+        d = blocks[:, d_off:d_off + 2].copy().view(np.float16).astype(np.float64).reshape(-1)
+        scale = np.repeat(d, per) if kind == "q5_0" else None
+        if kind == "q5_0":
+            q = (y.astype(np.float64) / np.where(scale == 0, 1, scale))
+            assert np.all(np.abs(q - np.round(q)) == 0) and q.min() >= -16 and q.max() <= 15
+        else:
+            sc = blocks[:, 192:208].view(np.int8).astype(np.float64)
+            a = np.repeat((d[:, None] * sc).reshape(-1), 16)
+            q = y.astype(np.float64) / np.where(a == 0, 1, a)
+            ok = a != 0
+            assert np.all(q[ok] == np.round(q[ok])) and q[ok].min() >= -32 and q[ok].max() <= 31
 
 
 # ----------------------------------------------------------- nearest code --
