@@ -51,8 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
-    ap.add_argument("--workload", choices=["step", "sweep", "llama"], default="step",
-                    help="step: the benchmark line; sweep / llama: informational tables")
+    ap.add_argument("--workload", choices=["step", "sweep", "llama", "gguf", "nested"], default="step",
+                    help="step: the benchmark line; sweep / llama / gguf / nested: informational tables")
     return ap.parse_args()
 
 
@@ -626,6 +626,75 @@ def run_llama(args):
           flush=True)
 
 
+def run_gguf(args):
+    """Every GGUF block type on two workloads, bf16 target: the Verification
+    table's 4096 blocks (fits in L2, so a 512 MiB flush precedes each
+    repetition and is subtracted) and a 4096 x 14336 weight matrix."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(1 << 29, dtype=torch.uint8, device=dev)
+    peak = measured_peaks()[0]
+    rows = []
+    for kind, (per, bb) in bq.GGUF_TYPES.items():
+        for label, nblk in (("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // per)):
+            blocks = torch.from_numpy(synth.gguf_blocks(nblk, kind, seed=9).reshape(-1)).to(dev)
+            y = torch.empty(nblk * per, dtype=torch.bfloat16, device=dev)
+            bq.dequant_gguf(kind, blocks, out=y)
+            ms = _timed(lambda: bq.dequant_gguf(kind, blocks, out=y), 50, flush)
+            nbytes = nblk * bb + 2 * per * nblk  # blocks read + bf16 written
+            rows.append({"type": kind, "workload": label, "blocks": nblk, "us": round(ms * 1e3, 2),
+                         "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
+                         "frac_of_measured_peak": round(nbytes / (ms / 1e3) / 1e9 / peak, 4)})
+            del blocks, y
+    print(json.dumps({"workload": "gguf", "target": "bf16", "rows": rows}), flush=True)
+
+
+def run_nested(args):
+    """Compressed statistics on the step's tensor (bf16 NF4 blocksize 64,
+    n = 2^29): the absmax array quantized again with the dynamic 8-bit table
+    in blocks of 256, then both dequantized; timed against the plain pair."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n = 1 << 29
+    x = synth.large_outliers()[0].to(dev)
+    nf4 = torch.from_numpy(codebooks.nf4()).to(dev)
+    dyn = torch.from_numpy(codebooks.dynamic8()).to(dev)
+    nb = n // BS
+    a = torch.empty(nb, dtype=torch.float32, device=dev)
+    q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    a2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    qa = torch.empty(nb, dtype=torch.uint8, device=dev)
+    a_back = torch.empty(nb, dtype=torch.float32, device=dev)
+    y = torch.empty(n, dtype=torch.bfloat16, device=dev)
+
+    def plain():
+        bq.quantize_blockwise(x, nf4, BS, absmax=a, out=q)
+        bq.dequantize_blockwise(q, a, n, BS, nf4, out=y)
+
+    def nested():
+        bq.quantize_blockwise(x, nf4, BS, absmax=a, out=q)
+        bq.quantize_blockwise(a, dyn, 256, absmax=a2, out=qa)
+        bq.dequantize_blockwise(qa, a2, nb, 256, dyn, out=a_back)
+        bq.dequantize_blockwise(q, a_back, n, BS, nf4, out=y)
+
+    for _ in range(3):
+        plain()
+        nested()
+    torch.cuda.synchronize()
+    reps = max(3, args.steps)
+    ms_plain = _timed(plain, reps)
+    ms_nested = _timed(nested, reps)
+    stats_plain = 4 * nb
+    stats_nested = nb + 4 * a2.numel()
+    print(json.dumps({"workload": "nested statistics, bf16 NF4 bs64 + dyn8 bs256 on absmax",
+                      "n": n, "plain_ms": round(ms_plain, 3), "nested_ms": round(ms_nested, 3),
+                      "overhead_pct": round(100 * (ms_nested / ms_plain - 1), 2),
+                      "stat_bytes_plain": stats_plain, "stat_bytes_nested": stats_nested,
+                      "bits_per_element_plain": round(4 + 8 * stats_plain / n, 4),
+                      "bits_per_element_nested": round(4 + 8 * stats_nested / n, 4)}),
+          flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_setup(args)
@@ -636,6 +705,10 @@ def main():
             run_sweep(args)
         elif args.workload == "llama":
             run_llama(args)
+        elif args.workload == "gguf":
+            run_gguf(args)
+        elif args.workload == "nested":
+            run_nested(args)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -1,5 +1,6 @@
-"""Blockwise codebook quantization / dequantization and GGUF Q8_0 / Q4_0
-dequantization on NVIDIA B200 (sm_100a).
+"""Blockwise codebook quantization / dequantization and GGUF block
+dequantization (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K) on NVIDIA B200
+(sm_100a).
 
 A thin ctypes binding over ``libbq.so`` (C ABI in ``include/bq.h``).  Every
 step of the computation runs in the library's CUDA kernels; this module only
@@ -20,10 +21,14 @@ LIB_PATH = os.path.join(_HERE, "libbq.so")
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_CUDA = 0, 1, 2, 3
 BQ_F32, BQ_F16, BQ_BF16 = 0, 1, 2
 
+# GGUF block types: (outputs per block, bytes per block)
+GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32, 22),
+              "q5_1": (32, 24), "q4_k": (256, 144), "q6_k": (256, 210)}
+
 EXPORTED = (
-    "bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
-    "bq_dequant_q4_0", "bq_status_string", "bq_last_cuda_error", "bq_device_fault",
-    "bq_abi_version",
+    "bq_quantize_blockwise", "bq_dequantize_blockwise",
+) + tuple("bq_dequant_" + k for k in GGUF_TYPES) + (
+    "bq_status_string", "bq_last_cuda_error", "bq_device_fault", "bq_abi_version",
 )
 
 _lib = None
@@ -49,10 +54,10 @@ def lib():
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
         L.bq_quantize_blockwise.argtypes = [vp, i32, i64, i32, vp, i32, vp, vp, vp]
         L.bq_dequantize_blockwise.argtypes = [vp, vp, i64, i32, vp, i32, vp, i32, vp]
-        L.bq_dequant_q8_0.argtypes = [vp, i64, vp, i32, vp]
-        L.bq_dequant_q4_0.argtypes = [vp, i64, vp, i32, vp]
-        for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
-                  "bq_dequant_q4_0", "bq_device_fault"):
+        for k in GGUF_TYPES:
+            getattr(L, "bq_dequant_" + k).argtypes = [vp, i64, vp, i32, vp]
+            getattr(L, "bq_dequant_" + k).restype = ctypes.c_int
+        for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_device_fault"):
             getattr(L, f).restype = ctypes.c_int
         L.bq_status_string.argtypes = [ctypes.c_int]
         L.bq_status_string.restype = ctypes.c_char_p
@@ -89,6 +94,26 @@ def bq_dequant_q8_0(blocks, n_blocks, y, y_dtype, stream):
 
 def bq_dequant_q4_0(blocks, n_blocks, y, y_dtype, stream):
     return lib().bq_dequant_q4_0(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q4_1(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q4_1(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q5_0(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q5_0(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q5_1(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q5_1(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q4_k(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q4_k(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q6_k(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q6_k(blocks, n_blocks, y, y_dtype, stream)
 
 
 def bq_status_string(status):
@@ -183,12 +208,20 @@ def dequantize_blockwise(q, absmax, n, blocksize, code, dtype=None, out=None, st
     return out
 
 
-def _gguf(fn, bbytes, blocks, dtype, out, stream):
+def dequant_gguf(kind, blocks, dtype=None, out=None, stream=None):
+    """GGUF blocks of type ``kind`` (a key of GGUF_TYPES; uint8 CUDA tensor of
+    n_blocks * block bytes) -> outputs-per-block * n_blocks values of ``dtype``
+    (default bf16)."""
     torch = _torch()
     _need_cuda(blocks, "blocks")
+    per, bbytes = GGUF_TYPES[kind]
+    if blocks.numel() % bbytes:
+        raise ValueError(f"{kind}: {blocks.numel()} bytes is not a whole number of "
+                         f"{bbytes}-byte blocks")
     nblk = blocks.numel() // bbytes
     if out is None:
-        out = torch.empty(32 * nblk, dtype=dtype or torch.bfloat16, device=blocks.device)
+        out = torch.empty(per * nblk, dtype=dtype or torch.bfloat16, device=blocks.device)
+    fn = globals()["bq_dequant_" + kind]
     _check(fn.__name__, fn(blocks.data_ptr(), nblk, out.data_ptr(), _dtype_code(out.dtype),
                            _stream_handle(stream)))
     return out
@@ -196,9 +229,59 @@ def _gguf(fn, bbytes, blocks, dtype, out, stream):
 
 def dequant_q8_0(blocks, dtype=None, out=None, stream=None):
     """GGUF Q8_0 blocks (uint8 CUDA tensor of n_blocks*34 bytes) -> 32*n_blocks values."""
-    return _gguf(bq_dequant_q8_0, 34, blocks, dtype, out, stream)
+    return dequant_gguf("q8_0", blocks, dtype, out, stream)
 
 
 def dequant_q4_0(blocks, dtype=None, out=None, stream=None):
     """GGUF Q4_0 blocks (uint8 CUDA tensor of n_blocks*18 bytes) -> 32*n_blocks values."""
-    return _gguf(bq_dequant_q4_0, 18, blocks, dtype, out, stream)
+    return dequant_gguf("q4_0", blocks, dtype, out, stream)
+
+
+def dequant_q4_1(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q4_1 blocks (n_blocks*20 bytes) -> 32*n_blocks values."""
+    return dequant_gguf("q4_1", blocks, dtype, out, stream)
+
+
+def dequant_q5_0(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q5_0 blocks (n_blocks*22 bytes) -> 32*n_blocks values."""
+    return dequant_gguf("q5_0", blocks, dtype, out, stream)
+
+
+def dequant_q5_1(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q5_1 blocks (n_blocks*24 bytes) -> 32*n_blocks values."""
+    return dequant_gguf("q5_1", blocks, dtype, out, stream)
+
+
+def dequant_q4_k(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q4_K super-blocks (n_blocks*144 bytes) -> 256*n_blocks values."""
+    return dequant_gguf("q4_k", blocks, dtype, out, stream)
+
+
+def dequant_q6_k(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q6_K super-blocks (n_blocks*210 bytes) -> 256*n_blocks values."""
+    return dequant_gguf("q6_k", blocks, dtype, out, stream)
+
+
+# -------------------------------------------------- compressed statistics ----
+
+def quantize_blockwise_nested(x, code, blocksize, code2, blocksize2=256, stream=None):
+    """Blockwise quantization with compressed statistics: the fp32 absmax array
+    of the first pass is itself quantized blockwise with `code2` (the dynamic
+    8-bit table) in blocks of `blocksize2`.  Two calls of the same C entry
+    point on the same stream.  Returns (codes, absmax codes, absmax2, absmax),
+    absmax being the first pass's fp32 statistics (kept by the caller only if
+    wanted)."""
+    absmax, q = quantize_blockwise(x, code, blocksize, stream=stream)
+    absmax2, qa = quantize_blockwise(absmax, code2, blocksize2, stream=stream)
+    return q, qa, absmax2, absmax
+
+
+def dequantize_blockwise_nested(q, qa, absmax2, n, blocksize, code, code2, blocksize2=256,
+                                dtype=None, stream=None):
+    """Inverse of quantize_blockwise_nested: the absmax array is dequantized to
+    fp32 first, then the elements."""
+    torch = _torch()
+    nb = (n + blocksize - 1) // blocksize
+    absmax = dequantize_blockwise(qa, absmax2, nb, blocksize2, code2, dtype=torch.float32,
+                                  stream=stream)
+    return dequantize_blockwise(q, absmax, n, blocksize, code, dtype=dtype, stream=stream)

@@ -208,7 +208,8 @@ bq_status launch_gguf(const bq::GParams& p, int dev, int sms, cudaStream_t strea
   int occ = 1;
   bq_status s = kernel_occupancy(slot, kernel, dev, bq::kGThreads, 0, &occ);
   if (s != BQ_OK) return s;
-  const int64_t steps = (p.n_blocks + bq::kGGroup * bq::kGUnroll - 1) / (bq::kGGroup * bq::kGUnroll);
+  constexpr int kStep = bq::GStep<KIND>::value;
+  const int64_t steps = (p.n_blocks + kStep - 1) / kStep;
   int64_t want = (steps + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   if (want > cap) want = cap;
@@ -344,6 +345,31 @@ bq_status bq_dequant_q8_0(const void* blocks, int64_t n_blocks, void* y, bq_dtyp
 bq_status bq_dequant_q4_0(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
                           cudaStream_t stream) {
   return gguf_entry<bq::kQ4_0>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q4_1(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ4_1>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q5_0(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ5_0>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q5_1(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ5_1>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q4_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ4_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q6_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ6_K>(blocks, n_blocks, y, y_dtype, stream);
 }
 
 const char* bq_status_string(bq_status s) {

@@ -1,23 +1,34 @@
-// bq_gguf.cuh - GGUF Q8_0 / Q4_0 dequantization (sm_100a).
+// bq_gguf.cuh - GGUF block dequantization (sm_100a): Q8_0, Q4_0, Q4_1, Q5_0,
+// Q5_1, Q4_K, Q6_K.
 //
-// Formats ("ComfyUI-GGUF PR #472, Cache device-side constants in dequant
-// kernels", Problem section and Verification table):
+// Formats.  Q8_0 and Q4_0 as on "ComfyUI-GGUF PR #472, Cache device-side
+// constants in dequant kernels", Problem section and Verification table:
 //   Q8_0 block = fp16 d + 32 signed bytes q:       y = d * q
 //   Q4_0 block = fp16 d + 16 bytes qs, shifts [0, 4]: y[j] = d * ((qs[j] & 15) - 8),
 //                                                    y[16 + j] = d * ((qs[j] >> 4) - 8)
-// The fp32 products are exact (an 11-bit d times |q| <= 128), so the narrowed
-// output is the correctly rounded value.  The page's point - no per-call
-// host-to-device constants - holds trivially here: the shift and offset live
-// in registers.
+// The other rows of that table follow the GGUF block layouts (the page names
+// the types without spelling them out):
+//   Q4_1 = fp16 d, fp16 m, qs[16]:            y = d * nibble + m
+//   Q5_0 = fp16 d, u32 qh, qs[16]:            y = d * (q - 16), q = nibble | bit e of qh << 4
+//   Q5_1 = fp16 d, fp16 m, u32 qh, qs[16]:    y = d * q + m
+//   Q4_K = super-block of 256: fp16 d, fp16 dmin, 12 bytes of packed 6-bit
+//          scales and mins for 8 sub-blocks of 32, qs[128]:  y = d*sc*q - dmin*mn
+//   Q6_K = super-block of 256: ql[128], qh[64], int8 scales[16], fp16 d:
+//          y = d * sc * (q - 32), q = 4 bits of ql | 2 bits of qh << 4
+// Every product here is exact in fp32 (an 11-bit d times at most 6 + 5 more
+// bits), so the only rounding before the narrowing is the add of a min,
+// done as one fma: the narrowed output is the correctly rounded value.  The
+// page's point - no per-call host-to-device constants - holds trivially here:
+// shifts and offsets live in registers.
 //
-// Kernel design.  A warp takes 4 groups of 8 blocks per step (32 blocks:
-// 1088 B for Q8_0, 576 B for Q4_0).  A group of 8 blocks is 272 or 144 bytes,
-// a whole number of 16-byte chunks, so in a 16-byte aligned stream every group
-// starts aligned and the warp stages its 4 groups into its shared buffer with
-// up to three 16-byte loads per lane, fetched into registers one step ahead.  Lane l
-// then decodes 8 outputs of block l/4 of each group and writes them as one
-// 16-byte store, so each warp store covers 512 contiguous bytes of bf16
-// output.  Bytes become floats with the 2^23 trick: a byte b placed in the low
+// Kernel design.  A lane always decodes 8 consecutive outputs of one block
+// and writes them as one 16-byte store (bf16), so a warp pass writes 512
+// contiguous bytes: 8 blocks of 32 (lanes 4b..4b+3 share block b) or one
+// super-block of 256.  A warp step covers 32 blocks (8 super-blocks), a whole
+// number of 16-byte chunks in every format, so in a 16-byte aligned stream
+// every step starts aligned; the warp stages a step into its shared buffer
+// with up to four 16-byte loads per lane, fetched into registers one step
+// ahead.  Bytes become floats with the 2^23 trick: a byte b placed in the low
 // mantissa bits of 2^23 is the float 2^23 + b, and subtracting 2^23 + offset
 // is exact.  Unaligned streams and the last partial step are staged byte by
 // byte.
@@ -27,7 +38,7 @@
 
 namespace bq {
 
-enum : int { kQ8_0 = 0, kQ4_0 = 1 };
+enum : int { kQ8_0 = 0, kQ4_0 = 1, kQ4_1 = 2, kQ5_0 = 3, kQ5_1 = 4, kQ4_K = 5, kQ6_K = 6 };
 
 struct GParams {
   const uint8_t* blocks;
@@ -37,12 +48,20 @@ struct GParams {
 };
 
 constexpr int kGThreads = 256;
-constexpr int kGGroup = 8;   // blocks per group (one warp-wide decode)
-constexpr int kGUnroll = 4;  // groups per warp step
 
+// BB: bytes per block; EPB: outputs per block; QS: offset of the nibble bytes;
+// QH: offset of the 32 high bits (Q5); MIN: the block carries an fp16 min
 template <int KIND> struct GTraits;
-template <> struct GTraits<kQ8_0> { static constexpr int BB = 34; };
-template <> struct GTraits<kQ4_0> { static constexpr int BB = 18; };
+template <> struct GTraits<kQ8_0> { static constexpr int BB = 34, EPB = 32, QS = 2, QH = 0; static constexpr bool MIN = false; };
+template <> struct GTraits<kQ4_0> { static constexpr int BB = 18, EPB = 32, QS = 2, QH = 0; static constexpr bool MIN = false; };
+template <> struct GTraits<kQ4_1> { static constexpr int BB = 20, EPB = 32, QS = 4, QH = 0; static constexpr bool MIN = true; };
+template <> struct GTraits<kQ5_0> { static constexpr int BB = 22, EPB = 32, QS = 6, QH = 2; static constexpr bool MIN = false; };
+template <> struct GTraits<kQ5_1> { static constexpr int BB = 24, EPB = 32, QS = 8, QH = 4; static constexpr bool MIN = true; };
+template <> struct GTraits<kQ4_K> { static constexpr int BB = 144, EPB = 256, QS = 16, QH = 0; static constexpr bool MIN = true; };
+template <> struct GTraits<kQ6_K> { static constexpr int BB = 210, EPB = 256, QS = 0, QH = 128; static constexpr bool MIN = false; };
+
+// blocks per warp step: 32 blocks of 32 or 8 super-blocks of 256
+template <int KIND> struct GStep { static constexpr int value = GTraits<KIND>::EPB == 32 ? 32 : 8; };
 
 // byte k of w placed in the low mantissa of 2^23: the float 2^23 + byte
 __device__ __forceinline__ float byte_as_float(uint32_t w, int k) {
@@ -62,34 +81,94 @@ __device__ __forceinline__ void load8_at2(const uint8_t* ptr, uint32_t& w0, uint
   w1 = __funnelshift_r(x1, x2, sh);
 }
 
-// Decode 8 outputs (part `part` of the block at bp) to narrowed words:
-// v = (float(2^23 + byte) - (2^23 + offset)) * d, two lanes per packed op.
-template <int KIND, int OT>
-__device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float (&v)[8]) {
-  const float d = __half2float(*reinterpret_cast<const __half*>(bp));
-  uint32_t w0, w1;
-  load8_at2(bp + 2 + (KIND == kQ8_0 ? 8 * part : 8 * (part & 1)), w0, w1);
-  float off;
-  if constexpr (KIND == kQ8_0) {
-    w0 ^= 0x80808080u;  // signed byte q -> q + 128
-    w1 ^= 0x80808080u;
-    off = 8388736.0f;   // 2^23 + 128
-  } else {
-    const int sh = (part >> 1) * 4;  // parts 0,1: low nibbles; 2,3: high nibbles
-    w0 = (w0 >> sh) & 0x0F0F0F0Fu;
-    w1 = (w1 >> sh) & 0x0F0F0F0Fu;
-    off = 8388616.0f;   // 2^23 + 8
-  }
-  const uint64_t o2 = pack2(-off, -off), d2 = pack2(d, d);
+__device__ __forceinline__ float half_at(const uint8_t* p) {
+  return __half2float(*reinterpret_cast<const __half*>(p));
+}
+
+// bit k (k < 4) of a nibble moved to bit 4 of byte k: the four shifted copies
+// x, x << 7, x << 14, x << 21 do not overlap, so the product is their OR
+__device__ __forceinline__ uint32_t spread4_to_bit4(uint32_t x4) {
+  return ((x4 * 0x00204081u) & 0x01010101u) << 4;
+}
+
+// v[k] = (float(2^23 + byte k) - (2^23 + off)) * s, or with a min:
+// fma(float(2^23 + byte k) - 2^23, s, m); two lanes per packed op
+template <bool MIN>
+__device__ __forceinline__ void bytes_to_values(uint32_t w0, uint32_t w1, float off, float s,
+                                                float m, float (&v)[8]) {
+  const uint64_t o2 = pack2(-off, -off), s2 = pack2(s, s), one2 = pack2(1.0f, 1.0f);
+  const uint64_t m2 = pack2(m, m);
 #pragma unroll
   for (int k = 0; k < 4; k += 2) {
     // x - off as fma(x, 1, -off): one rounding, exact here
-    const uint64_t a = fma2(pack2(byte_as_float(w0, k), byte_as_float(w0, k + 1)),
-                            pack2(1.0f, 1.0f), o2);
-    const uint64_t b = fma2(pack2(byte_as_float(w1, k), byte_as_float(w1, k + 1)),
-                            pack2(1.0f, 1.0f), o2);
-    unpack2(mul2(a, d2), v[k], v[k + 1]);
-    unpack2(mul2(b, d2), v[4 + k], v[4 + k + 1]);
+    const uint64_t a = fma2(pack2(byte_as_float(w0, k), byte_as_float(w0, k + 1)), one2, o2);
+    const uint64_t b = fma2(pack2(byte_as_float(w1, k), byte_as_float(w1, k + 1)), one2, o2);
+    if constexpr (MIN) {
+      unpack2(fma2(a, s2, m2), v[k], v[k + 1]);
+      unpack2(fma2(b, s2, m2), v[4 + k], v[4 + k + 1]);
+    } else {
+      unpack2(mul2(a, s2), v[k], v[k + 1]);
+      unpack2(mul2(b, s2), v[4 + k], v[4 + k + 1]);
+    }
+  }
+}
+
+// Decode outputs 8*part .. 8*part+7 of the block at bp (part < EPB / 8).
+template <int KIND>
+__device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float (&v)[8]) {
+  using T = GTraits<KIND>;
+  uint32_t w0, w1;
+  if constexpr (KIND == kQ8_0) {
+    load8_at2(bp + 2 + 8 * part, w0, w1);
+    w0 ^= 0x80808080u;  // signed byte q -> q + 128
+    w1 ^= 0x80808080u;
+    bytes_to_values<false>(w0, w1, 8388736.0f /* 2^23 + 128 */, half_at(bp), 0.0f, v);
+  } else if constexpr (T::EPB == 32) {
+    // nibble formats: parts 0, 1 are the low nibbles of qs[0..7], qs[8..15];
+    // parts 2, 3 the high nibbles
+    load8_at2(bp + T::QS + 8 * (part & 1), w0, w1);
+    const int sh = (part >> 1) * 4;
+    w0 = (w0 >> sh) & 0x0F0F0F0Fu;
+    w1 = (w1 >> sh) & 0x0F0F0F0Fu;
+    if constexpr (T::QH != 0) {
+      const uint32_t hb = bp[T::QH + part];  // bits 8*part .. 8*part+7 of qh
+      w0 |= spread4_to_bit4(hb & 15u);
+      w1 |= spread4_to_bit4(hb >> 4);
+    }
+    const float d = half_at(bp);
+    if constexpr (T::MIN) {
+      bytes_to_values<true>(w0, w1, 8388608.0f /* 2^23 */, d, half_at(bp + 2), v);
+    } else {
+      const float off = KIND == kQ4_0 ? 8388616.0f /* 2^23 + 8 */ : 8388624.0f /* 2^23 + 16 */;
+      bytes_to_values<false>(w0, w1, off, d, 0.0f, v);
+    }
+  } else if constexpr (KIND == kQ4_K) {
+    // part = 8g + 4h + r: group g of 64 reads qs[32g + 8r ..], nibble half h,
+    // sub-block 2g + h
+    const int g = part >> 3, h = (part >> 2) & 1, r = part & 3;
+    const int is = 2 * g + h, j = is & 3;
+    const uint32_t A = bp[4 + j], B = bp[8 + j], C = bp[12 + j];
+    const bool hi = is >= 4;
+    const uint32_t sc = hi ? ((C & 15u) | ((A >> 6) << 4)) : (A & 63u);
+    const uint32_t mn = hi ? ((C >> 4) | ((B >> 6) << 4)) : (B & 63u);
+    const float a = half_at(bp) * static_cast<float>(sc);        // exact
+    const float b = half_at(bp + 2) * static_cast<float>(mn);    // exact
+    const uint2 q = *reinterpret_cast<const uint2*>(bp + 16 + 32 * g + 8 * r);  // 8-byte aligned
+    w0 = (q.x >> (4 * h)) & 0x0F0F0F0Fu;
+    w1 = (q.y >> (4 * h)) & 0x0F0F0F0Fu;
+    bytes_to_values<true>(w0, w1, 8388608.0f, a, -b, v);
+  } else {  // kQ6_K
+    // part = 16n + 4c + r: half n, 32-element chunk c, outputs 8r..8r+7 of it
+    const int n = part >> 4, c = (part >> 2) & 3, r = part & 3;
+    uint32_t h0, h1;
+    load8_at2(bp + 64 * n + 32 * (c & 1) + 8 * r, w0, w1);
+    load8_at2(bp + 128 + 32 * n + 8 * r, h0, h1);
+    const int sl = 4 * (c >> 1), sh = 2 * c;
+    w0 = ((w0 >> sl) & 0x0F0F0F0Fu) | (((h0 >> sh) & 0x03030303u) << 4);
+    w1 = ((w1 >> sl) & 0x0F0F0F0Fu) | (((h1 >> sh) & 0x03030303u) << 4);
+    const int scale = static_cast<int8_t>(bp[192 + 8 * n + (r >> 1) + 2 * c]);
+    const float a = half_at(bp + 208) * static_cast<float>(scale);  // exact
+    bytes_to_values<false>(w0, w1, 8388640.0f /* 2^23 + 32 */, a, 0.0f, v);
   }
 }
 
@@ -115,13 +194,18 @@ __device__ __forceinline__ void store8(void* y, int64_t e0, const float (&v)[8],
 
 template <int KIND, int OT>
 __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
-  constexpr int BB = GTraits<KIND>::BB;
-  constexpr int STEP_BLOCKS = kGGroup * kGUnroll;  // 32
-  constexpr int STEP_BYTES = STEP_BLOCKS * BB;     // 1088 or 576, multiples of 16
-  constexpr int STEP_CHUNKS = STEP_BYTES / 16;     // 68 or 36
-  constexpr int LOADS = (STEP_CHUNKS + 31) / 32;   // per lane: 3 or 2
-  // 16 bytes of padding: the 8-byte reads of the last block load one aligned
-  // word past the block
+  using T = GTraits<KIND>;
+  constexpr int BB = T::BB;
+  constexpr int LPB = T::EPB / 8;                  // lanes per block: 4 or 32
+  constexpr int GROUP = 32 / LPB;                  // blocks per warp pass: 8 or 1
+  constexpr int STEP_BLOCKS = GStep<KIND>::value;
+  constexpr int UNROLL = STEP_BLOCKS / GROUP;      // warp passes per step: 4 or 8
+  constexpr int STEP_BYTES = STEP_BLOCKS * BB;     // a multiple of 16 in every format
+  constexpr int STEP_CHUNKS = STEP_BYTES / 16;
+  constexpr int LOADS = (STEP_CHUNKS + 31) / 32;   // per lane: 2 to 4
+  static_assert(STEP_BYTES % 16 == 0, "a step must be whole 16-byte chunks");
+  // 16 bytes of padding: the 8-byte reads of the last block may load one
+  // aligned word past the block
   __shared__ __align__(16) uint8_t buf[kGThreads / 32][STEP_BYTES + 16];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,14 +247,14 @@ __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
     }
     __syncwarp();
 
-    const int part = lane & 3;
+    const int part = lane % LPB;
 #pragma unroll
-    for (int u = 0; u < kGUnroll; ++u) {
-      const int bl = u * kGGroup + (lane >> 2);
+    for (int u = 0; u < UNROLL; ++u) {
+      const int bl = u * GROUP + lane / LPB;
       if (bl < nblk) {
         float v[8];
-        gguf_decode8<KIND, OT>(wb + bl * BB, part, v);
-        store8<OT>(p.y, (blk0 + bl) * 32 + part * 8, v, p.vec != 0);
+        gguf_decode8<KIND>(wb + bl * BB, part, v);
+        store8<OT>(p.y, (blk0 + bl) * T::EPB + part * 8, v, p.vec != 0);
       }
     }
     __syncwarp();

@@ -1,6 +1,7 @@
 /*
- * bq.h - blockwise codebook quantization / dequantization and GGUF
- * Q8_0 / Q4_0 dequantization on NVIDIA B200 (sm_100a).  C ABI of libbq.so.
+ * bq.h - blockwise codebook quantization / dequantization and GGUF block
+ * dequantization (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K) on NVIDIA B200
+ * (sm_100a).  C ABI of libbq.so.
  *
  * Common contract of every compute entry point
  * -------------------------------------------
@@ -124,6 +125,60 @@ BQ_API bq_status bq_dequant_q8_0(const void *blocks, int64_t n_blocks, void *y,
  *   y        device, 32 * n_blocks elements of y_dtype, written.
  */
 BQ_API bq_status bq_dequant_q4_0(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * The other block types of the same page's Verification table (Q4_1, Q5_0,
+ * Q5_1, Q4_K, Q6_K: 4096 blocks, bf16 target, bit-identical across
+ * implementations).  The page names them without spelling out their bytes;
+ * these entry points follow the GGUF block layouts below.  All fp16 fields are
+ * little endian; every product is exact in fp32, so the output is the
+ * correctly rounded value of the formula, the min being added once.
+ * Arguments as for bq_dequant_q8_0: blocks are device bytes (any alignment),
+ * y receives (elements per block) * n_blocks values of y_dtype.
+ *
+ * Q4_1: 20-byte blocks {fp16 d, fp16 m, qs[16]}, 32 outputs:
+ *   y[32k + j] = d * (qs[j] & 15) + m,  y[32k + 16 + j] = d * (qs[j] >> 4) + m
+ */
+BQ_API bq_status bq_dequant_q4_1(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q5_0: 22-byte blocks {fp16 d, uint32 qh, qs[16]}, 32 outputs: output e
+ * takes its low 4 bits as in Q4_0 and bit e of qh as bit 4 (q in 0..31):
+ *   y[32k + e] = d * (q - 16)
+ */
+BQ_API bq_status bq_dequant_q5_0(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q5_1: 24-byte blocks {fp16 d, fp16 m, uint32 qh, qs[16]}, q as in Q5_0:
+ *   y[32k + e] = d * q + m
+ */
+BQ_API bq_status bq_dequant_q5_1(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q4_K: 144-byte super-blocks {fp16 d, fp16 dmin, scales[12], qs[128]}, 256
+ * outputs in 8 sub-blocks of 32.  Sub-block i < 4 has scale scales[i] & 63 and
+ * min scales[i + 4] & 63; i >= 4 has scale (scales[i + 4] & 15) |
+ * (scales[i - 4] >> 6) << 4 and min (scales[i + 4] >> 4) | (scales[i] >> 6) << 4.
+ * Group g (outputs 64g .. 64g + 63) reads qs[32g .. 32g + 31]: low nibbles
+ * are sub-block 2g, high nibbles sub-block 2g + 1.
+ *   y = d * scale * q - dmin * min
+ */
+BQ_API bq_status bq_dequant_q4_k(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q6_K: 210-byte super-blocks {ql[128], qh[64], int8 scales[16], fp16 d}, 256
+ * outputs in 16 sub-blocks of 16 (sub-block j uses scales[j]).  In half n
+ * (outputs 128n ..), output 32c + l (c < 4, l < 32) takes its low 4 bits from
+ * ql[64n + 32(c & 1) + l] (low nibble for c < 2, else high) and bits 4..5
+ * from bits 2c, 2c + 1 of qh[32n + l]:
+ *   y = d * scales[j] * (q - 32)
+ */
+BQ_API bq_status bq_dequant_q6_k(const void *blocks, int64_t n_blocks, void *y,
                           bq_dtype y_dtype, cudaStream_t stream);
 
 /* Static text for a status code. */

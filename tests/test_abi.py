@@ -23,16 +23,18 @@ def L():
     return bq.lib()
 
 
-def test_header_declares_the_four_calls():
+def test_header_declares_the_compute_calls():
     syms = declared_symbols()
     for name in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
-                 "bq_dequant_q4_0"):
+                 "bq_dequant_q4_0", "bq_dequant_q4_1", "bq_dequant_q5_0", "bq_dequant_q5_1",
+                 "bq_dequant_q4_k", "bq_dequant_q6_k"):
         assert name in syms
 
 
 def test_every_declared_symbol_is_exported(L):
     syms = declared_symbols()
-    assert len(syms) >= 8
+    assert len(syms) >= 13
+    assert set(syms) == set(bq.EXPORTED)
     for name in syms:
         assert hasattr(L, name), name
         assert name in bq.EXPORTED
@@ -78,6 +80,15 @@ def test_rejects_bad_sizes_pointers_dtypes(L):
     assert bq.bq_dequant_q4_0(0, 10, P, bq.BQ_BF16, 0) == E
     assert bq.bq_dequant_q4_0(P, 10, P + 1, bq.BQ_BF16, 0) == E
     assert bq.bq_dequant_q4_0(P, 10, P, 9, 0) == E
+    for kind in bq.GGUF_TYPES:
+        fn = getattr(bq, "bq_dequant_" + kind)
+        assert fn(P, -1, P, bq.BQ_BF16, 0) == E, kind
+        assert fn(0, 10, P, bq.BQ_BF16, 0) == E, kind
+        assert fn(P, 10, 0, bq.BQ_BF16, 0) == E, kind
+        assert fn(P, 10, P + 1, bq.BQ_F16, 0) == E, kind
+        assert fn(P, 10, P + 2, bq.BQ_F32, 0) == E, kind
+        assert fn(P, 10, P, 3, 0) == E, kind
+        assert fn(P, 1 << 53, P, bq.BQ_BF16, 0) == E, kind
 
 
 def test_zero_length_is_ok_without_touching_the_device(L):
@@ -86,6 +97,8 @@ def test_zero_length_is_ok_without_touching_the_device(L):
     assert bq.bq_dequantize_blockwise(0, 0, 0, 64, 0, 256, 0, bq.BQ_BF16, 0) == bq.BQ_OK
     assert bq.bq_dequant_q8_0(0, 0, 0, bq.BQ_BF16, 0) == bq.BQ_OK
     assert bq.bq_dequant_q4_0(0, 0, 0, bq.BQ_F32, 0) == bq.BQ_OK
+    for kind in bq.GGUF_TYPES:
+        assert getattr(bq, "bq_dequant_" + kind)(0, 0, 0, bq.BQ_BF16, 0) == bq.BQ_OK, kind
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

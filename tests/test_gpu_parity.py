@@ -231,34 +231,50 @@ def test_ordering_case_detects_wrong_stream():
 
 # ------------------------------------------------------------------ GGUF --
 
-@pytest.mark.parametrize("kind", ["q8_0", "q4_0"])
+@pytest.mark.parametrize("kind", list(bq.GGUF_TYPES))
 @pytest.mark.parametrize("ydtype", ["bf16", "f16", "f32"])
 def test_gguf_parity(kind, ydtype):
-    bb = 34 if kind == "q8_0" else 18
-    fn = bq.bq_dequant_q8_0 if kind == "q8_0" else bq.bq_dequant_q4_0
-    ofn = oracle.dequant_q8_0 if kind == "q8_0" else oracle.dequant_q4_0
-    for nblk, off in ((4096, 0), (4096 * 14336 // 32, 0), (1, 0), (7, 0), (8, 0), (9, 0),
+    """Every output of every block, bit for bit, on random blocks: sizes that
+    span many warp steps (the 4096 x 14336 matrix among them), partial steps,
+    single blocks, and streams at byte offsets 1, 2 and 16."""
+    per, bb = bq.GGUF_TYPES[kind]
+    fn = getattr(bq, "bq_dequant_" + kind)
+    for nblk, off in ((4096, 0), (4096 * 14336 // per, 0), (1, 0), (7, 0), (8, 0), (9, 0),
                       (1000 + 3, 0), (1003, 2), (517, 1), (64, 16)):
         blocks = synth.gguf_blocks(nblk, kind, seed=4 + nblk)
         bt, bp = device_copy(blocks, off)
-        y = Guarded(EB[ydtype] * 32 * nblk)
+        y = Guarded(EB[ydtype] * per * nblk)
         assert fn(bp, nblk, y.ptr, DT_CODE[ydtype], 0) == bq.BQ_OK
         torch.cuda.synchronize()
         assert y.guards_intact()
         got = y.host().view(np.float32 if ydtype == "f32" else np.uint16)
-        want = ofn(blocks, ydtype)
+        want = oracle.dequant_gguf(kind, blocks, ydtype)
         assert np.array_equal(got, want), (kind, nblk, off)
 
 
 def test_gguf_hand_blocks_on_gpu():
     import test_oracle_pins as pins
     for kind, blk, expect in pins._load_hand_blocks():
-        fn = bq.bq_dequant_q8_0 if kind == "q8_0" else bq.bq_dequant_q4_0
+        per, _ = bq.GGUF_TYPES[kind]
+        fn = getattr(bq, "bq_dequant_" + kind)
         bt, bp = device_copy(blk)
-        y = Guarded(4 * 32)
+        y = Guarded(4 * per)
         assert fn(bp, 1, y.ptr, bq.BQ_F32, 0) == bq.BQ_OK
         torch.cuda.synchronize()
-        assert np.array_equal(y.host().view(np.uint32), expect.view(np.uint32))
+        assert np.array_equal(y.host().view(np.uint32), expect.view(np.uint32)), kind
+
+
+def test_gguf_torch_helpers():
+    """The torch-level helpers: output sizes, default dtype and whole-block check."""
+    for kind, (per, bb) in bq.GGUF_TYPES.items():
+        blocks = synth.gguf_blocks(33, kind, seed=77)
+        t = torch.from_numpy(blocks.reshape(-1)).cuda()
+        y = bq.dequant_gguf(kind, t)
+        assert y.dtype == torch.bfloat16 and y.numel() == 33 * per
+        want = oracle.dequant_gguf(kind, blocks, "bf16")
+        assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), want)
+        with pytest.raises(ValueError):
+            bq.dequant_gguf(kind, t[:-1])
 
 
 # ------------------------------------------------------ full-size configs --
@@ -387,3 +403,29 @@ def test_bounded_wait_gives_up_and_context_survives(probes):
     # the context is still healthy: a normal quantize call works
     x = small_input(8192 * 2 + 5, "bf16", 64, seed=1)
     check_quant(x, "bf16", 64, "nf4")
+
+
+# ------------------------------------------------- compressed statistics ---
+
+@pytest.mark.parametrize("dtype,bs", [("bf16", 64), ("f16", 4096), ("f32", 32)])
+def test_nested_statistics_parity(dtype, bs):
+    """Compressed statistics: the absmax array quantized with the dynamic
+    8-bit table in blocks of 256, against the same composition of oracle
+    calls."""
+    n = 300 * bs + 37
+    x = synth.with_zero_block(synth.normal(n, dtype, seed=bs + 1), bs)
+    nf4, dyn = TABLES["nf4"], TABLES["dyn8"]
+    q, qa, a2, a = bq.quantize_blockwise_nested(x.cuda(), code_dev(nf4), bs, code_dev(dyn))
+    y = bq.dequantize_blockwise_nested(q, qa, a2, n, bs, code_dev(nf4), code_dev(dyn),
+                                       dtype=x.dtype)
+    torch.cuda.synchronize()
+    xh = np_bits(x)
+    oa, oq = oracle.quantize_blockwise(xh, dtype, bs, nf4)
+    oa2, oqa = oracle.quantize_blockwise(oa, "f32", 256, dyn)
+    oa_back = oracle.dequantize_blockwise(oqa, oa2, oa.size, 256, dyn, "f32")
+    oy = oracle.dequantize_blockwise(oq, oa_back, n, bs, nf4, dtype)
+    assert np.array_equal(a.cpu().numpy(), oa)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(qa.cpu().numpy(), oqa)
+    assert np.array_equal(a2.cpu().numpy(), oa2)
+    assert np.array_equal(np_bits(y.cpu()), oy)
