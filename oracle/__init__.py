@@ -57,6 +57,10 @@ def _declare(L):
     L.bqo_dequant_q8_0.restype = c_int
     L.bqo_dequant_q4_0.argtypes = [c_void_p, c_int64, c_void_p, c_int]
     L.bqo_dequant_q4_0.restype = c_int
+    for kind in ("q8_0", "q4_0"):
+        f = getattr(L, "bqo_quantize_" + kind)
+        f.argtypes = [c_void_p, c_int, c_int64, c_void_p]
+        f.restype = c_int
     for kind in GGUF_TYPES:
         f = getattr(L, "bqo_dequant_" + kind)
         f.argtypes = [c_void_p, c_int64, c_void_p, c_int]
@@ -155,6 +159,18 @@ def dequant_gguf(kind, blocks, ydtype, L=None):
     if getattr(L, "bqo_dequant_" + kind)(_ptr(blocks), nblk, _ptr(y), DTYPES[ydtype]) != 0:
         raise ValueError("oracle rejected the arguments")
     return y
+
+
+def quantize_gguf(kind, x, dtype, L=None):
+    """Encode x (n a multiple of 32) as GGUF Q8_0 or Q4_0 blocks
+    (uint8 array [n / 32, block bytes])."""
+    L = L or lib()
+    per, bb = GGUF_TYPES[kind]
+    xb = _as_bits(x, dtype).reshape(-1)
+    out = np.empty((xb.size // 32, bb), np.uint8)
+    if getattr(L, "bqo_quantize_" + kind)(_ptr(xb), DTYPES[dtype], xb.size, _ptr(out)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
 
 
 def nearest_code(xn, code, L=None):

@@ -354,3 +354,76 @@ int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
     }
     return 0;
 }
+
+/* ------------------------------------------------------- GGUF encoders -- */
+
+static void put_half(uint8_t *p, float v)
+{
+    uint16_t h = bqo_f32_to_f16(v);
+    p[0] = (uint8_t)(h & 0xff);
+    p[1] = (uint8_t)(h >> 8);
+}
+
+int bqo_quantize_q8_0(const void *x, int dtype, int64_t n, uint8_t *blocks)
+{
+    if (n < 0 || n % 32 != 0 || !valid_dtype(dtype))
+        return -1;
+    for (int64_t k = 0; k < n / 32; ++k) {
+        float amax = 0.0f;
+        for (int j = 0; j < 32; ++j)
+            amax = fmaxf(amax, fabsf(load_elem(x, dtype, 32 * k + j)));
+        float d = amax / 127.0f;
+        float id = (d == 0.0f) ? 0.0f : 1.0f / d;
+        uint8_t *blk = blocks + 34 * k;
+        put_half(blk, d);
+        for (int j = 0; j < 32; ++j) {
+            float r = roundf(load_elem(x, dtype, 32 * k + j) * id);
+            int q;
+            if (r >= 127.0f)
+                q = 127;
+            else if (r <= -127.0f)
+                q = -127;
+            else if (r == r)
+                q = (int)r;
+            else
+                q = 0;
+            blk[2 + j] = (uint8_t)(int8_t)q;
+        }
+    }
+    return 0;
+}
+
+int bqo_quantize_q4_0(const void *x, int dtype, int64_t n, uint8_t *blocks)
+{
+    if (n < 0 || n % 32 != 0 || !valid_dtype(dtype))
+        return -1;
+    for (int64_t k = 0; k < n / 32; ++k) {
+        /* the element of largest magnitude, first on ties; starting below
+         * every magnitude takes element 0 unless it is NaN */
+        float amax = -1.0f, m = 0.0f;
+        for (int j = 0; j < 32; ++j) {
+            float v = load_elem(x, dtype, 32 * k + j);
+            if (fabsf(v) > amax) {
+                amax = fabsf(v);
+                m = v;
+            }
+        }
+        float d = m / -8.0f;
+        float id = (d == 0.0f) ? 0.0f : 1.0f / d;
+        uint8_t *blk = blocks + 18 * k;
+        put_half(blk, d);
+        int q[32];
+        for (int j = 0; j < 32; ++j) {
+            float t = truncf(load_elem(x, dtype, 32 * k + j) * id + 8.5f);
+            if (t >= 15.0f)
+                q[j] = 15;
+            else if (t >= 0.0f)
+                q[j] = (int)t;
+            else
+                q[j] = 0;
+        }
+        for (int j = 0; j < 16; ++j)
+            blk[2 + j] = (uint8_t)(q[j] | (q[j + 16] << 4));
+    }
+    return 0;
+}

@@ -96,6 +96,26 @@ int bqo_dequant_q4_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
  * the 6-bit value (4 low bits from ql, 2 high bits from qh). */
 int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
 
+/*
+ * GGUF encoders (the inverse direction of Q8_0 / Q4_0), following the GGUF
+ * format's reference quantizer.  x holds n elements (n a multiple of 32) of
+ * element type dtype; blocks receives n / 32 blocks.  All arithmetic is fp32
+ * on the exactly widened input.
+ *
+ * Q8_0: amax = max |x| over the block (NaN ignored), d = amax / 127,
+ * id = (d == 0 ? 0 : 1 / d), q_j = round-half-away(x_j * id), then clamped
+ * to [-127, 127] (only non-finite values reach the clamp; NaN gives 0);
+ * the block stores fp16(d) (round to nearest even) and the q_j as int8.
+ *
+ * Q4_0: m = the element of largest |x| (the first one on ties, NaN never
+ * chosen, +0 if every element is NaN), d = m / -8, id = (d == 0 ? 0 : 1 / d),
+ * t_j = trunc(x_j * id + 8.5), q_j = 15 if t_j >= 15, else t_j if t_j >= 0,
+ * else 0 (NaN gives 0); byte j = q_j | q_(j+16) << 4; the block stores fp16(d).
+ * Returns 0, or -1 on a bad argument.
+ */
+int bqo_quantize_q8_0(const void *x, int dtype, int64_t n, uint8_t *blocks);
+int bqo_quantize_q4_0(const void *x, int dtype, int64_t n, uint8_t *blocks);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,14 @@ MUTANTS = [
     ("q6k_offset", "int q = (lo4 | (hi2 << 4)) - 32;", "int q = (lo4 | (hi2 << 4)) - 31;"),
     ("q6k_scale_index", "sc[8 * n + l / 16 + 2 * c]", "sc[8 * n + l / 16 + c]"),
     ("q6k_qh_shift", "int hi2 = (qh[32 * n + l] >> (2 * c)) & 3;", "int hi2 = (qh[32 * n + l] >> c) & 3;"),
+    ("q8_enc_divisor", "float d = amax / 127.0f;", "float d = amax / 128.0f;"),
+    ("q8_enc_round_half_even", "float r = roundf(load_elem(x, dtype, 32 * k + j) * id);",
+     "float r = rintf(load_elem(x, dtype, 32 * k + j) * id);"),
+    ("q4_enc_last_tie_wins", "if (fabsf(v) > amax) {", "if (fabsf(v) >= amax) {"),
+    ("q4_enc_abs_max", "float d = m / -8.0f;", "float d = amax / -8.0f;"),
+    ("q4_enc_no_half", "* id + 8.5f);", "* id + 8.0f);"),
+    ("q4_enc_nibble_order", "blk[2 + j] = (uint8_t)(q[j] | (q[j + 16] << 4));",
+     "blk[2 + j] = (uint8_t)((q[j] << 4) | q[j + 16]);"),
     ("f16_bias", "ldexpf((float)(m + 1024), e - 25)", "ldexpf((float)(m + 1024), e - 24)"),
     ("bf16_ties_away", "if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))",
      "if (lower >= 0x8000u)"),
@@ -69,6 +77,8 @@ def _all_pins():
         pins.test_f32_to_bf16_matches_torch_rne,
         pins.test_gguf_hand_worked_blocks,
         pins.test_gguf_matches_gguf_package,
+        pins.test_gguf_encode_hand_worked_blocks,
+        pins.test_gguf_encode_matches_gguf_package,
         pins.test_nearest_code_ties_go_low,
         pins.test_quantize_hand_worked_packing,
         lambda: pins.test_nearest_code_brute_force("nf4"),

@@ -183,6 +183,78 @@ def test_gguf_more_types_exact_products():
             assert np.all(q[ok] == np.round(q[ok])) and q[ok].min() >= -32 and q[ok].max() <= 31
 
 
+# ---------------------------------------------------------- GGUF encoders --
+
+def _load_encode_blocks():
+    recs = []
+    with open(os.path.join(GOLDEN, "gguf_encode_blocks.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            blk = np.frombuffer(bytes.fromhex(parts[1]), np.uint8)
+            x = np.array([float(v) for v in parts[2:]], np.float32)
+            recs.append((parts[0], blk, x))
+    return recs
+
+
+def test_gguf_encode_hand_worked_blocks():
+    recs = _load_encode_blocks()
+    assert len(recs) == 7
+    for kind, blk, x in recs:
+        assert x.size == 32 and blk.size == oracle.GGUF_TYPES[kind][1]
+        for dt, xv in (("f32", x), ("f16", x.astype(np.float16)),
+                       ("bf16", torch.from_numpy(x).to(torch.bfloat16).view(torch.int16)
+                        .numpy().view(np.uint16))):
+            got = oracle.quantize_gguf(kind, xv, dt).reshape(-1)
+            assert np.array_equal(got, blk), (kind, dt, got.tobytes().hex())
+
+
+def test_gguf_encode_matches_gguf_package():
+    """Independent cross-check: the gguf package's quantizer (bit-exact with
+    the format's reference implementation), on normal data, data with many
+    ties, zero blocks (one starting with -0), bf16 input widened."""
+    gq = pytest.importorskip("gguf.quants")
+    import gguf
+    T = gguf.GGMLQuantizationType
+    g = torch.Generator().manual_seed(31)
+    base = torch.randn(32 * 4096, generator=g).mul_(0.02)
+    cases = [base.numpy(), (base * 1000).round().numpy()]
+    z = base.numpy().copy()
+    z[:64] = 0.0
+    z[64:96] = -0.0
+    z[128] = -0.0
+    z[129:160] = 0.0
+    cases.append(z)
+    for kind, qt in (("q8_0", T.Q8_0), ("q4_0", T.Q4_0)):
+        for x in cases:
+            x = np.ascontiguousarray(x, np.float32)
+            ref = gq.quantize(x.reshape(-1, 32), qt)
+            assert np.array_equal(oracle.quantize_gguf(kind, x, "f32"), ref), kind
+        xb = base.to(torch.bfloat16)
+        ref = gq.quantize(xb.float().numpy().reshape(-1, 32), qt)
+        got = oracle.quantize_gguf(kind, xb.view(torch.int16).numpy().view(np.uint16), "bf16")
+        assert np.array_equal(got, ref), kind
+
+
+def test_gguf_encode_round_trip_bound():
+    """Decoding an encoded block lands within the format's step of the input:
+    |x - d*q| <= |d|/2 (Q8_0) and <= |d| (Q4_0, truncation after +8.5 can lose
+    up to one step at the clamp), d being the stored fp16 scale, up to the fp16
+    rounding of d times |q|."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(32 * 2048, generator=g).mul_(0.02).numpy()
+    for kind, step in (("q8_0", 0.5), ("q4_0", 1.0)):
+        blocks = oracle.quantize_gguf(kind, x, "f32")
+        y = oracle.dequant_gguf(kind, blocks, "f32").astype(np.float64)
+        d = np.abs(blocks[:, :2].copy().view(np.float16).astype(np.float64)).reshape(-1)
+        dd = np.repeat(d, 32)
+        # fp16 rounding of d moves every output by at most |q| * ulp16(d) / 2
+        slack = 16 * dd * 2.0 ** -10 if kind == "q4_0" else 127 * dd * 2.0 ** -10
+        assert np.all(np.abs(x - y) <= step * dd + slack + 1e-12), kind
+
+
 # ----------------------------------------------------------- nearest code --
 
 def _exact_nearest(xn, table):
