@@ -646,6 +646,20 @@ def run_gguf(args):
                          "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
                          "frac_of_measured_peak": round(nbytes / (ms / 1e3) / 1e9 / peak, 4)})
             del blocks, y
+    # the encoders, bf16 input of the same two sizes
+    for kind in bq.GGUF_ENCODERS:
+        bb = bq.GGUF_TYPES[kind][1]
+        for label, nblk in (("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // 32)):
+            g = torch.Generator(device=dev)
+            g.manual_seed(17)
+            x = torch.randn(nblk * 32, generator=g, device=dev).mul_(0.02).to(torch.bfloat16)
+            out = bq.quantize_gguf(kind, x)
+            ms = _timed(lambda: bq.quantize_gguf(kind, x, out=out), 50, flush)
+            nbytes = nblk * (64 + bb)  # bf16 read + blocks written
+            rows.append({"type": kind + " encode", "workload": label, "blocks": nblk,
+                         "us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
+                         "frac_of_measured_peak": round(nbytes / (ms / 1e3) / 1e9 / peak, 4)})
+            del x, out
     print(json.dumps({"workload": "gguf", "target": "bf16", "rows": rows}), flush=True)
 
 

@@ -25,9 +25,12 @@ BQ_F32, BQ_F16, BQ_BF16 = 0, 1, 2
 GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32, 22),
               "q5_1": (32, 24), "q4_k": (256, 144), "q6_k": (256, 210)}
 
+GGUF_ENCODERS = ("q8_0", "q4_0")
+
 EXPORTED = (
     "bq_quantize_blockwise", "bq_dequantize_blockwise",
-) + tuple("bq_dequant_" + k for k in GGUF_TYPES) + (
+) + tuple("bq_dequant_" + k for k in GGUF_TYPES) + tuple(
+    "bq_quantize_" + k for k in GGUF_ENCODERS) + (
     "bq_status_string", "bq_last_cuda_error", "bq_device_fault", "bq_abi_version",
 )
 
@@ -57,6 +60,9 @@ def lib():
         for k in GGUF_TYPES:
             getattr(L, "bq_dequant_" + k).argtypes = [vp, i64, vp, i32, vp]
             getattr(L, "bq_dequant_" + k).restype = ctypes.c_int
+        for k in GGUF_ENCODERS:
+            getattr(L, "bq_quantize_" + k).argtypes = [vp, i32, i64, vp, vp]
+            getattr(L, "bq_quantize_" + k).restype = ctypes.c_int
         for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_device_fault"):
             getattr(L, f).restype = ctypes.c_int
         L.bq_status_string.argtypes = [ctypes.c_int]
@@ -114,6 +120,14 @@ def bq_dequant_q4_k(blocks, n_blocks, y, y_dtype, stream):
 
 def bq_dequant_q6_k(blocks, n_blocks, y, y_dtype, stream):
     return lib().bq_dequant_q6_k(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_quantize_q8_0(x, x_dtype, n, blocks, stream):
+    return lib().bq_quantize_q8_0(x, x_dtype, n, blocks, stream)
+
+
+def bq_quantize_q4_0(x, x_dtype, n, blocks, stream):
+    return lib().bq_quantize_q4_0(x, x_dtype, n, blocks, stream)
 
 
 def bq_status_string(status):
@@ -260,6 +274,26 @@ def dequant_q4_k(blocks, dtype=None, out=None, stream=None):
 def dequant_q6_k(blocks, dtype=None, out=None, stream=None):
     """GGUF Q6_K super-blocks (n_blocks*210 bytes) -> 256*n_blocks values."""
     return dequant_gguf("q6_k", blocks, dtype, out, stream)
+
+
+def quantize_gguf(kind, x, out=None, stream=None):
+    """Encode the CUDA tensor x (fp32/fp16/bf16, numel a multiple of 32) as
+    GGUF ``kind`` blocks ("q8_0" or "q4_0"): a uint8 tensor of
+    numel/32 * block bytes."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    if kind not in GGUF_ENCODERS:
+        raise ValueError(f"no encoder for {kind}")
+    n = x.numel()
+    if n % 32:
+        raise ValueError(f"{n} elements is not a whole number of 32-element blocks")
+    bbytes = GGUF_TYPES[kind][1]
+    if out is None:
+        out = torch.empty(n // 32 * bbytes, dtype=torch.uint8, device=x.device)
+    fn = globals()["bq_quantize_" + kind]
+    _check(fn.__name__, fn(x.data_ptr(), _dtype_code(x.dtype), n, out.data_ptr(),
+                           _stream_handle(stream)))
+    return out
 
 
 # -------------------------------------------------- compressed statistics ----

@@ -14,6 +14,7 @@
 
 #include "bq_dequant.cuh"
 #include "bq_gguf.cuh"
+#include "bq_gguf_encode.cuh"
 #include "bq_quantize.cuh"
 
 static_assert(int(BQ_F32) == int(bq::kF32) && int(BQ_F16) == int(bq::kF16) &&
@@ -242,6 +243,46 @@ bq_status gguf_entry(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_d
   }
 }
 
+template <int KIND, int IT>
+bq_status launch_gguf_encode(const bq::GEParams& p, int dev, int sms, cudaStream_t stream) {
+  static KernelSlot slot;
+  auto kernel = bq::gguf_encode_kernel<KIND, IT>;
+  int occ = 1;
+  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kGThreads, 0, &occ);
+  if (s != BQ_OK) return s;
+  const int64_t steps = (p.n_blocks + 31) / 32;
+  int64_t want = (steps + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
+  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kGThreads, 0, stream, p);
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "gguf encode launch");
+}
+
+template <int KIND>
+bq_status gguf_encode_entry(const void* x, bq_dtype x_dtype, int64_t n, void* blocks,
+                            cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || n % 32 != 0 || !valid_dtype(x_dtype)) return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (n > (int64_t{1} << 50)) return BQ_ERR_INVALID_ARG;
+  if (!x || !blocks || !aligned(x, elem_bytes(x_dtype))) return BQ_ERR_INVALID_ARG;
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+  bq::GEParams p;
+  p.x = x;
+  p.blocks = static_cast<uint8_t*>(blocks);
+  p.n_blocks = n / 32;
+  p.vec = aligned(x, 16) && aligned(blocks, 16);
+  switch (x_dtype) {
+    case BQ_F32: return launch_gguf_encode<KIND, bq::kF32>(p, dev, info.sms, stream);
+    case BQ_F16: return launch_gguf_encode<KIND, bq::kF16>(p, dev, info.sms, stream);
+    default: return launch_gguf_encode<KIND, bq::kBF16>(p, dev, info.sms, stream);
+  }
+}
+
 }  // namespace
 
 // ===================================================================== ABI ==
@@ -370,6 +411,16 @@ bq_status bq_dequant_q4_k(const void* blocks, int64_t n_blocks, void* y, bq_dtyp
 bq_status bq_dequant_q6_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
                           cudaStream_t stream) {
   return gguf_entry<bq::kQ6_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_quantize_q8_0(const void* x, bq_dtype x_dtype, int64_t n, void* blocks,
+                           cudaStream_t stream) {
+  return gguf_encode_entry<bq::kQ8_0>(x, x_dtype, n, blocks, stream);
+}
+
+bq_status bq_quantize_q4_0(const void* x, bq_dtype x_dtype, int64_t n, void* blocks,
+                           cudaStream_t stream) {
+  return gguf_encode_entry<bq::kQ4_0>(x, x_dtype, n, blocks, stream);
 }
 
 const char* bq_status_string(bq_status s) {

@@ -181,6 +181,31 @@ BQ_API bq_status bq_dequant_q4_k(const void *blocks, int64_t n_blocks, void *y,
 BQ_API bq_status bq_dequant_q6_k(const void *blocks, int64_t n_blocks, void *y,
                           bq_dtype y_dtype, cudaStream_t stream);
 
+/*
+ * GGUF Q8_0 / Q4_0 encoders: the inverse direction of bq_dequant_q8_0 and
+ * bq_dequant_q4_0 (same page: the Problem section and Verification table
+ * give the block formats, not an encoder).  They follow the GGUF format's
+ * reference quantizer, in fp32 on the exactly widened input:
+ *   Q8_0: d = max|x| / 127, id = (d == 0 ? 0 : 1/d),
+ *         q_j = round-half-away(x_j * id); block = fp16(d), int8 q[32]
+ *   Q4_0: m = the element of largest |x| (the first on ties), d = m / -8,
+ *         id = (d == 0 ? 0 : 1/d), q_j = min(15, trunc(x_j * id + 8.5));
+ *         block = fp16(d), byte j = q_j | q_(j+16) << 4
+ * fp16(d) rounds to nearest even.  Non-finite inputs are clamped (Q8_0 to
+ * [-127, 127], Q4_0 to [0, 15], NaN to 0; NaN never chosen as m), so every
+ * input gives defined bytes.
+ *   x        device, n elements of x_dtype (aligned to the element size);
+ *            n must be a multiple of 32 (GGUF rows are whole blocks).
+ *   blocks   device, (n / 32) * 34 (Q8_0) or * 18 (Q4_0) bytes, written
+ *            (any byte alignment).
+ * BQ_ERR_INVALID_ARG for n < 0, n % 32 != 0, a bad dtype, null or misaligned
+ * pointers; n == 0 returns BQ_OK without a launch.
+ */
+BQ_API bq_status bq_quantize_q8_0(const void *x, bq_dtype x_dtype, int64_t n, void *blocks,
+                                  cudaStream_t stream);
+BQ_API bq_status bq_quantize_q4_0(const void *x, bq_dtype x_dtype, int64_t n, void *blocks,
+                                  cudaStream_t stream);
+
 /* Static text for a status code. */
 BQ_API const char *bq_status_string(bq_status s);
 

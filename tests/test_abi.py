@@ -27,13 +27,13 @@ def test_header_declares_the_compute_calls():
     syms = declared_symbols()
     for name in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
                  "bq_dequant_q4_0", "bq_dequant_q4_1", "bq_dequant_q5_0", "bq_dequant_q5_1",
-                 "bq_dequant_q4_k", "bq_dequant_q6_k"):
+                 "bq_dequant_q4_k", "bq_dequant_q6_k", "bq_quantize_q8_0", "bq_quantize_q4_0"):
         assert name in syms
 
 
 def test_every_declared_symbol_is_exported(L):
     syms = declared_symbols()
-    assert len(syms) >= 13
+    assert len(syms) >= 15
     assert set(syms) == set(bq.EXPORTED)
     for name in syms:
         assert hasattr(L, name), name
@@ -89,6 +89,17 @@ def test_rejects_bad_sizes_pointers_dtypes(L):
         assert fn(P, 10, P + 2, bq.BQ_F32, 0) == E, kind
         assert fn(P, 10, P, 3, 0) == E, kind
         assert fn(P, 1 << 53, P, bq.BQ_BF16, 0) == E, kind
+    for kind in bq.GGUF_ENCODERS:
+        fn = getattr(bq, "bq_quantize_" + kind)
+        assert fn(P, bq.BQ_BF16, -32, P, 0) == E, kind
+        assert fn(P, bq.BQ_BF16, 33, P, 0) == E, kind       # not whole blocks
+        assert fn(P, bq.BQ_BF16, 48, P, 0) == E, kind
+        assert fn(0, bq.BQ_BF16, 64, P, 0) == E, kind
+        assert fn(P, bq.BQ_BF16, 64, 0, 0) == E, kind
+        assert fn(P + 1, bq.BQ_BF16, 64, P, 0) == E, kind
+        assert fn(P + 2, bq.BQ_F32, 64, P, 0) == E, kind
+        assert fn(P, 5, 64, P, 0) == E, kind
+        assert fn(P, bq.BQ_F32, 1 << 51, P, 0) == E, kind
 
 
 def test_zero_length_is_ok_without_touching_the_device(L):
@@ -99,6 +110,8 @@ def test_zero_length_is_ok_without_touching_the_device(L):
     assert bq.bq_dequant_q4_0(0, 0, 0, bq.BQ_F32, 0) == bq.BQ_OK
     for kind in bq.GGUF_TYPES:
         assert getattr(bq, "bq_dequant_" + kind)(0, 0, 0, bq.BQ_BF16, 0) == bq.BQ_OK, kind
+    for kind in bq.GGUF_ENCODERS:
+        assert getattr(bq, "bq_quantize_" + kind)(0, bq.BQ_BF16, 0, 0, 0) == bq.BQ_OK, kind
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -277,6 +277,97 @@ def test_gguf_torch_helpers():
             bq.dequant_gguf(kind, t[:-1])
 
 
+# --------------------------------------------------------- GGUF encoders --
+
+def _encode_input(nblk, dtype, seed, special=False):
+    """N(0, 0.02) blocks, with every 7th block rounded to a grid of 1/64
+    (ties on |x| and exact halves after scaling) and every 11th all zeros
+    (every 22nd starting with -0).  `special` adds blocks with inf, -inf,
+    NaN, fp32/bf16 subnormals and magnitudes whose scale reciprocal
+    overflows."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(nblk, 32, generator=g).mul_(0.02)
+    x[::7] = torch.round(x[::7] * 64) / 64
+    x[::11] = 0.0
+    x[::22, 0] = -0.0
+    if special:
+        x[1::13, 3] = float("inf")
+        x[2::13, 5] = -float("inf")
+        x[3::13, 0] = float("nan")
+        x[4::13, :] = float("nan")
+        x[5::13, :] *= 2.0 ** -120           # d subnormal, 1/d overflows
+        x[6::13, 9] = 2.0 ** -133            # bf16-representable subnormal maximum ...
+        x[6::13, :9] = 0.0
+        x[6::13, 10:] = 0.0
+        x[7::13, :] = torch.tensor(1e-40)    # fp32 subnormal everywhere
+        x[8::13, 4] = 65504.0 * 4            # beyond fp16 range: d overflows fp16
+    return x.reshape(-1).to(synth.TORCH_DTYPES[dtype])
+
+
+@pytest.mark.parametrize("kind", ["q8_0", "q4_0"])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_gguf_encode_parity(kind, dtype):
+    """Every byte of every block against the oracle: many warp steps (the
+    4096 x 14336 matrix among them), partial steps, single blocks, inputs at
+    element offsets that break 16-byte alignment, outputs at byte offsets."""
+    bb = bq.GGUF_TYPES[kind][1]
+    fn = getattr(bq, "bq_quantize_" + kind)
+    for nblk, xoff, ooff in ((4096, 0, 0), (4096 * 14336 // 32, 0, 0), (1, 0, 0), (31, 0, 0),
+                             (32, 0, 0), (33, 0, 0), (1003, 1, 3), (517, 0, 1), (64, 8, 16),
+                             (200, 3, 0)):
+        x = _encode_input(nblk, dtype, seed=nblk + xoff)
+        xh = np_bits(x)
+        xt, xp = device_copy(xh, xoff * EB[dtype])
+        out = Guarded(nblk * bb, offset=ooff)
+        assert fn(xp, DT_CODE[dtype], 32 * nblk, out.ptr, 0) == bq.BQ_OK
+        torch.cuda.synchronize()
+        assert out.guards_intact()
+        want = oracle.quantize_gguf(kind, xh, dtype).reshape(-1)
+        got = out.host()
+        assert np.array_equal(got, want), (kind, dtype, nblk, xoff, ooff,
+                                           int(np.nonzero(got != want)[0][0]) // bb)
+
+
+@pytest.mark.parametrize("kind", ["q8_0", "q4_0"])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_gguf_encode_special_values(kind, dtype):
+    """Non-finite and subnormal inputs: the clamps give the same defined
+    bytes on both sides."""
+    nblk = 13 * 40
+    x = _encode_input(nblk, dtype, seed=99, special=True)
+    xh = np_bits(x)
+    blocks = bq.quantize_gguf(kind, x.cuda())
+    want = oracle.quantize_gguf(kind, xh, dtype).reshape(-1)
+    assert np.array_equal(blocks.cpu().numpy(), want)
+
+
+def test_gguf_encode_hand_blocks_and_round_trip():
+    import test_oracle_pins as pins
+    for kind, blk, x in pins._load_encode_blocks():
+        for dt in ("f32", "f16", "bf16"):
+            t = torch.from_numpy(x).to(synth.TORCH_DTYPES[dt]).cuda()
+            assert np.array_equal(bq.quantize_gguf(kind, t).cpu().numpy(), blk), (kind, dt)
+    # encode -> decode on the device equals the oracle's encode -> decode
+    x = _encode_input(4096, "bf16", seed=5).cuda()
+    for kind in ("q8_0", "q4_0"):
+        y = bq.dequant_gguf(kind, bq.quantize_gguf(kind, x))
+        want = oracle.dequant_gguf(kind, oracle.quantize_gguf(kind, np_bits(x), "bf16"), "bf16")
+        assert np.array_equal(np_bits(y), want)
+
+
+def test_gguf_encode_rejects_bad_arguments():
+    x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(2 * 34, dtype=torch.uint8, device="cuda")
+    E = bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_quantize_q8_0(x.data_ptr(), bq.BQ_BF16, 63, out.data_ptr(), 0) == E
+    assert bq.bq_quantize_q4_0(x.data_ptr() + 1, bq.BQ_BF16, 32, out.data_ptr(), 0) == E
+    with pytest.raises(ValueError):
+        bq.quantize_gguf("q8_0", x[:40])
+    with pytest.raises(ValueError):
+        bq.quantize_gguf("q4_k", x)
+    assert bq.bq_device_fault() == 0
+
+
 # ------------------------------------------------------ full-size configs --
 
 def _run_full(x_cpu, dtype, bs, name, sample=3000, seed=0):
