@@ -51,8 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
-    ap.add_argument("--workload", choices=["step", "sweep", "llama", "gguf", "nested"], default="step",
-                    help="step: the benchmark line; sweep / llama / gguf / nested: informational tables")
+    ap.add_argument("--workload", choices=["step", "sweep", "llama", "gguf", "nested", "h2d"], default="step",
+                    help="step: the benchmark line; the others: informational tables")
     return ap.parse_args()
 
 
@@ -678,7 +678,6 @@ def run_nested(args):
     q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
     a2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
     qa = torch.empty(nb, dtype=torch.uint8, device=dev)
-    a_back = torch.empty(nb, dtype=torch.float32, device=dev)
     y = torch.empty(n, dtype=torch.bfloat16, device=dev)
 
     def plain():
@@ -686,10 +685,23 @@ def run_nested(args):
         bq.dequantize_blockwise(q, a, n, BS, nf4, out=y)
 
     def nested():
+        bq.quantize_blockwise_nested(x, nf4, BS, dyn, 256, absmax=a, out=q, absmax2=a2,
+                                     qabsmax=qa)
+        bq.dequantize_blockwise_nested(q, qa, a2, n, BS, nf4, dyn, 256, out=y)
+
+    def nested_parts():
+        # the same four kernels timed apart: two quantize passes, the fused
+        # dequantization
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
         bq.quantize_blockwise(x, nf4, BS, absmax=a, out=q)
+        e[1].record()
         bq.quantize_blockwise(a, dyn, 256, absmax=a2, out=qa)
-        bq.dequantize_blockwise(qa, a2, nb, 256, dyn, out=a_back)
-        bq.dequantize_blockwise(q, a_back, n, BS, nf4, out=y)
+        e[2].record()
+        bq.dequantize_blockwise_nested(q, qa, a2, n, BS, nf4, dyn, 256, out=y)
+        e[3].record()
+        torch.cuda.synchronize()
+        return [e[i].elapsed_time(e[i + 1]) for i in range(3)]
 
     for _ in range(3):
         plain()
@@ -698,14 +710,76 @@ def run_nested(args):
     reps = max(3, args.steps)
     ms_plain = _timed(plain, reps)
     ms_nested = _timed(nested, reps)
+    parts = [sorted(x) [len(x) // 2] for x in zip(*[nested_parts() for _ in range(reps)])]
     stats_plain = 4 * nb
     stats_nested = nb + 4 * a2.numel()
     print(json.dumps({"workload": "nested statistics, bf16 NF4 bs64 + dyn8 bs256 on absmax",
                       "n": n, "plain_ms": round(ms_plain, 3), "nested_ms": round(ms_nested, 3),
                       "overhead_pct": round(100 * (ms_nested / ms_plain - 1), 2),
+                      "nested_parts_ms": {"quantize": round(parts[0], 4),
+                                          "quantize_statistics": round(parts[1], 4),
+                                          "dequantize_fused": round(parts[2], 4)},
                       "stat_bytes_plain": stats_plain, "stat_bytes_nested": stats_nested,
                       "bits_per_element_plain": round(4 + 8 * stats_plain / n, 4),
                       "bits_per_element_nested": round(4 + 8 * stats_nested / n, 4)}),
+          flush=True)
+
+
+def run_h2d(args):
+    """Host input to quantized device output, bf16 NF4 bs64 with compressed
+    statistics (dyn8, blocks of 256), n = 2^28 in pinned host memory: the
+    serialized form (copy everything, then quantize on one stream - the
+    baseline of the bnb page's two-stream pipeline cells) against the
+    two-stream chunked pipeline at several chunk sizes.  GB/s of host input."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n = 1 << 28
+    g = torch.Generator().manual_seed(11)
+    x = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+    for lo in range(0, n, 1 << 24):
+        x[lo:lo + (1 << 24)] = torch.randn(1 << 24, generator=g).mul_(0.02).to(torch.bfloat16)
+    nf4 = torch.from_numpy(codebooks.nf4()).to(dev)
+    dyn = torch.from_numpy(codebooks.dynamic8()).to(dev)
+    xd = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    nb = n // BS
+    a = torch.empty(nb, dtype=torch.float32, device=dev)
+    q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    a2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    qa = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def serial():
+        xd.copy_(x, non_blocking=True)
+        bq.quantize_blockwise_nested(xd, nf4, BS, dyn, 256, absmax=a, out=q, absmax2=a2, qabsmax=qa)
+
+    reps = max(3, args.steps)
+    rows = []
+    for _ in range(2):
+        serial()
+    torch.cuda.synchronize()
+    ms = _timed(serial, reps)
+    rows.append({"form": "serial", "ms": round(ms, 3), "gbs": round(2 * n / (ms / 1e3) / 1e9, 2)})
+    ref = (q.clone(), qa.clone(), a2.clone())
+    for chunk in (1 << 22, 1 << 23, 1 << 24, 1 << 25):
+        staging = torch.empty(2 * chunk * 2, dtype=torch.uint8, device=dev)
+        side = torch.cuda.Stream(device=dev)
+        cur = torch.cuda.current_stream(dev)
+
+        def piped():
+            side.wait_stream(cur)
+            st = bq.bq_quantize_blockwise_host(
+                x.data_ptr(), bq.BQ_BF16, n, BS, nf4.data_ptr(), 16, dyn.data_ptr(), 256, 256,
+                a.data_ptr(), q.data_ptr(), a2.data_ptr(), qa.data_ptr(), staging.data_ptr(),
+                staging.numel(), chunk, cur.cuda_stream, side.cuda_stream)
+            assert st == bq.BQ_OK
+
+        q.zero_()
+        piped()
+        torch.cuda.synchronize()
+        same = bool(torch.equal(q, ref[0]) and torch.equal(qa, ref[1]) and torch.equal(a2, ref[2]))
+        ms = _timed(piped, reps)
+        rows.append({"form": "two-stream pipeline", "chunk_elements": chunk, "ms": round(ms, 3),
+                     "gbs": round(2 * n / (ms / 1e3) / 1e9, 2), "identical_to_serial": same})
+    print(json.dumps({"workload": "h2d + nested NF4 quantize, bf16 n=2^28 pinned", "rows": rows}),
           flush=True)
 
 
@@ -723,6 +797,8 @@ def main():
             run_gguf(args)
         elif args.workload == "nested":
             run_nested(args)
+        elif args.workload == "h2d":
+            run_h2d(args)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -28,7 +28,8 @@ GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32,
 GGUF_ENCODERS = ("q8_0", "q4_0")
 
 EXPORTED = (
-    "bq_quantize_blockwise", "bq_dequantize_blockwise",
+    "bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_quantize_blockwise_nested",
+    "bq_dequantize_blockwise_nested", "bq_quantize_blockwise_host",
 ) + tuple("bq_dequant_" + k for k in GGUF_TYPES) + tuple(
     "bq_quantize_" + k for k in GGUF_ENCODERS) + (
     "bq_status_string", "bq_last_cuda_error", "bq_device_fault", "bq_abi_version",
@@ -63,7 +64,15 @@ def lib():
         for k in GGUF_ENCODERS:
             getattr(L, "bq_quantize_" + k).argtypes = [vp, i32, i64, vp, vp]
             getattr(L, "bq_quantize_" + k).restype = ctypes.c_int
-        for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_device_fault"):
+        L.bq_quantize_blockwise_nested.argtypes = [vp, i32, i64, i32, vp, i32, vp, i32, i32, vp,
+                                                   vp, vp, vp, vp]
+        L.bq_dequantize_blockwise_nested.argtypes = [vp, vp, vp, i64, i32, vp, i32, vp, i32, i32,
+                                                     vp, i32, vp]
+        L.bq_quantize_blockwise_host.argtypes = [vp, i32, i64, i32, vp, i32, vp, i32, i32, vp, vp,
+                                                 vp, vp, vp, i64, i64, vp, vp]
+        for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_device_fault",
+                  "bq_quantize_blockwise_nested", "bq_dequantize_blockwise_nested",
+                  "bq_quantize_blockwise_host"):
             getattr(L, f).restype = ctypes.c_int
         L.bq_status_string.argtypes = [ctypes.c_int]
         L.bq_status_string.restype = ctypes.c_char_p
@@ -92,6 +101,29 @@ def bq_quantize_blockwise(x, x_dtype, n, blocksize, code, code_entries, absmax, 
 def bq_dequantize_blockwise(q, absmax, n, blocksize, code, code_entries, y, y_dtype, stream):
     return lib().bq_dequantize_blockwise(q, absmax, n, blocksize, code, code_entries, y, y_dtype,
                                          stream)
+
+
+def bq_quantize_blockwise_nested(x, x_dtype, n, blocksize, code, code_entries, code2,
+                                 code2_entries, blocksize2, absmax, out, absmax2, qabsmax, stream):
+    return lib().bq_quantize_blockwise_nested(x, x_dtype, n, blocksize, code, code_entries, code2,
+                                              code2_entries, blocksize2, absmax, out, absmax2,
+                                              qabsmax, stream)
+
+
+def bq_dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code, code_entries, code2,
+                                   code2_entries, blocksize2, y, y_dtype, stream):
+    return lib().bq_dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code,
+                                                code_entries, code2, code2_entries, blocksize2, y,
+                                                y_dtype, stream)
+
+
+def bq_quantize_blockwise_host(x_host, x_dtype, n, blocksize, code, code_entries, code2,
+                               code2_entries, blocksize2, absmax, out, absmax2, qabsmax, staging,
+                               staging_bytes, chunk_elements, stream0, stream1):
+    return lib().bq_quantize_blockwise_host(x_host, x_dtype, n, blocksize, code, code_entries,
+                                            code2, code2_entries, blocksize2, absmax, out,
+                                            absmax2, qabsmax, staging, staging_bytes,
+                                            chunk_elements, stream0, stream1)
 
 
 def bq_dequant_q8_0(blocks, n_blocks, y, y_dtype, stream):
@@ -298,24 +330,92 @@ def quantize_gguf(kind, x, out=None, stream=None):
 
 # -------------------------------------------------- compressed statistics ----
 
-def quantize_blockwise_nested(x, code, blocksize, code2, blocksize2=256, stream=None):
+def quantize_blockwise_nested(x, code, blocksize, code2, blocksize2=256, absmax=None, out=None,
+                              absmax2=None, qabsmax=None, stream=None):
     """Blockwise quantization with compressed statistics: the fp32 absmax array
-    of the first pass is itself quantized blockwise with `code2` (the dynamic
-    8-bit table) in blocks of `blocksize2`.  Two calls of the same C entry
-    point on the same stream.  Returns (codes, absmax codes, absmax2, absmax),
-    absmax being the first pass's fp32 statistics (kept by the caller only if
-    wanted)."""
-    absmax, q = quantize_blockwise(x, code, blocksize, stream=stream)
-    absmax2, qa = quantize_blockwise(absmax, code2, blocksize2, stream=stream)
-    return q, qa, absmax2, absmax
-
-
-def dequantize_blockwise_nested(q, qa, absmax2, n, blocksize, code, code2, blocksize2=256,
-                                dtype=None, stream=None):
-    """Inverse of quantize_blockwise_nested: the absmax array is dequantized to
-    fp32 first, then the elements."""
+    of the first pass is itself quantized blockwise with `code2` (the 256-entry
+    dynamic 8-bit table) in blocks of `blocksize2`.  Returns (codes, absmax
+    codes, absmax2, absmax), absmax being the first pass's fp32 statistics."""
     torch = _torch()
+    _need_cuda(x, "x")
+    _need_cuda(code, "code")
+    _need_cuda(code2, "code2")
+    n = x.numel()
     nb = (n + blocksize - 1) // blocksize
-    absmax = dequantize_blockwise(qa, absmax2, nb, blocksize2, code2, dtype=torch.float32,
-                                  stream=stream)
-    return dequantize_blockwise(q, absmax, n, blocksize, code, dtype=dtype, stream=stream)
+    dev = x.device
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty(code_bytes(n, code.numel()), dtype=torch.uint8, device=dev)
+    if absmax2 is None:
+        absmax2 = torch.empty((nb + blocksize2 - 1) // blocksize2, dtype=torch.float32, device=dev)
+    if qabsmax is None:
+        qabsmax = torch.empty(nb, dtype=torch.uint8, device=dev)
+    _check("bq_quantize_blockwise_nested", bq_quantize_blockwise_nested(
+        x.data_ptr(), _dtype_code(x.dtype), n, blocksize, code.data_ptr(), code.numel(),
+        code2.data_ptr(), code2.numel(), blocksize2, absmax.data_ptr(), out.data_ptr(),
+        absmax2.data_ptr(), qabsmax.data_ptr(), _stream_handle(stream)))
+    return out, qabsmax, absmax2, absmax
+
+
+def dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code, code2, blocksize2=256,
+                                dtype=None, out=None, stream=None):
+    """Inverse of quantize_blockwise_nested in one launch: each block's scale
+    is rebuilt from its code and the second-level scale inside the kernel."""
+    torch = _torch()
+    for t, name in ((q, "q"), (qabsmax, "qabsmax"), (absmax2, "absmax2"), (code, "code"),
+                    (code2, "code2")):
+        _need_cuda(t, name)
+    if out is None:
+        out = torch.empty(n, dtype=dtype or torch.bfloat16, device=q.device)
+    _check("bq_dequantize_blockwise_nested", bq_dequantize_blockwise_nested(
+        q.data_ptr(), qabsmax.data_ptr(), absmax2.data_ptr(), n, blocksize, code.data_ptr(),
+        code.numel(), code2.data_ptr(), code2.numel(), blocksize2, out.data_ptr(),
+        _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+# ------------------------------------------------------ host-input pipeline ----
+
+_side_streams = {}
+
+
+def quantize_blockwise_host(x_host, code, blocksize, code2=None, blocksize2=256,
+                            chunk_elements=1 << 24, staging=None, device=None):
+    """Quantize a CPU tensor (pin it for overlap) straight into device outputs,
+    copying and quantizing chunk by chunk over two streams: torch's current
+    stream and a side stream, joined back into the current stream.  Returns
+    (absmax, codes) or, with code2, (codes, absmax codes, absmax2, absmax)
+    like quantize_blockwise_nested."""
+    torch = _torch()
+    if x_host.is_cuda or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous CPU tensor")
+    dev = torch.device(device) if device is not None else torch.device(
+        "cuda", torch.cuda.current_device())
+    n = x_host.numel()
+    nb = (n + blocksize - 1) // blocksize
+    eb = x_host.element_size()
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    out = torch.empty(code_bytes(n, code.numel()), dtype=torch.uint8, device=dev)
+    absmax2 = qabsmax = None
+    if code2 is not None:
+        absmax2 = torch.empty((nb + blocksize2 - 1) // blocksize2, dtype=torch.float32, device=dev)
+        qabsmax = torch.empty(nb, dtype=torch.uint8, device=dev)
+    chunks = max(1, (n + chunk_elements - 1) // chunk_elements)
+    need = 2 * chunk_elements * eb if chunks > 1 else max(n, 1) * eb
+    if staging is None:
+        staging = torch.empty(need, dtype=torch.uint8, device=dev)
+    cur = torch.cuda.current_stream(dev)
+    side = _side_streams.get(dev.index)
+    if side is None:
+        side = _side_streams[dev.index] = torch.cuda.Stream(device=dev)
+    side.wait_stream(cur)  # outputs and staging were made on the current stream
+    _check("bq_quantize_blockwise_host", bq_quantize_blockwise_host(
+        x_host.data_ptr(), _dtype_code(x_host.dtype), n, blocksize, code.data_ptr(), code.numel(),
+        code2.data_ptr() if code2 is not None else None, 256, blocksize2, absmax.data_ptr(),
+        out.data_ptr(), absmax2.data_ptr() if absmax2 is not None else None,
+        qabsmax.data_ptr() if qabsmax is not None else None, staging.data_ptr(),
+        staging.numel(), chunk_elements, cur.cuda_stream, side.cuda_stream))
+    if code2 is None:
+        return absmax, out
+    return out, qabsmax, absmax2, absmax

@@ -178,10 +178,10 @@ bq_status dispatch_quantize(const bq::QParams& p, int entries, const CUtensorMap
 
 // ----------------------------------------------------------- dequantize ---
 
-template <int E, int OT>
+template <int E, int OT, bool NESTED>
 bq_status launch_dequant(const bq::DParams& p, int dev, int sms, cudaStream_t stream) {
   static KernelSlot slot;
-  auto kernel = bq::dequant_kernel<E, OT>;
+  auto kernel = bq::dequant_kernel<E, OT, NESTED>;
   int occ = 1;
   bq_status s = kernel_occupancy(slot, kernel, dev, bq::kDThreads, 0, &occ);
   if (s != BQ_OK) return s;
@@ -194,10 +194,33 @@ bq_status launch_dequant(const bq::DParams& p, int dev, int sms, cudaStream_t st
   return e == cudaSuccess ? BQ_OK : cuda_fail(e, "dequantize launch");
 }
 
-template <int OT>
+template <int OT, bool NESTED>
 bq_status dispatch_dequant(const bq::DParams& p, int entries, int dev, int sms, cudaStream_t st) {
-  if (entries == 16) return launch_dequant<16, OT>(p, dev, sms, st);
-  return launch_dequant<256, OT>(p, dev, sms, st);
+  if (entries == 16) return launch_dequant<16, OT, NESTED>(p, dev, sms, st);
+  return launch_dequant<256, OT, NESTED>(p, dev, sms, st);
+}
+
+// Shared by the plain and the compressed-statistics dequantization: p.q,
+// p.absmax or (p.qa, p.absmax2, p.code2, p.bs2_log2), p.code and p.y are set
+// and validated by the caller.
+template <bool NESTED>
+bq_status dequant_entry(bq::DParams p, int64_t n, int32_t blocksize, int32_t code_entries,
+                        bq_dtype y_dtype, cudaStream_t stream) {
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+  p.n = n;
+  p.bs_log2 = log2i(blocksize);
+  const int ce = 16 / elem_bytes(y_dtype);
+  const int qb = code_entries == 16 ? ce / 2 : ce;
+  p.vec = aligned(p.y, 16) && aligned(p.q, qb);
+  p.nchunks = p.vec ? n / ce : 0;
+  switch (y_dtype) {
+    case BQ_F32: return dispatch_dequant<bq::kF32, NESTED>(p, code_entries, dev, info.sms, stream);
+    case BQ_F16: return dispatch_dequant<bq::kF16, NESTED>(p, code_entries, dev, info.sms, stream);
+    default: return dispatch_dequant<bq::kBF16, NESTED>(p, code_entries, dev, info.sms, stream);
+  }
 }
 
 // ----------------------------------------------------------------- GGUF ---
@@ -354,28 +377,129 @@ bq_status bq_dequantize_blockwise(const uint8_t* q, const float* absmax, int64_t
   if (!q || !absmax || !code || !y || !aligned(absmax, 4) || !aligned(code, 4) ||
       !aligned(y, elem_bytes(y_dtype)))
     return BQ_ERR_INVALID_ARG;
-
-  int dev;
-  DevInfo info;
-  bq_status s = current_device(&dev, &info);
-  if (s != BQ_OK) return s;
-
-  bq::DParams p;
+  bq::DParams p{};
   p.q = q;
   p.absmax = absmax;
   p.code = code;
   p.y = y;
-  p.n = n;
-  p.bs_log2 = log2i(blocksize);
-  const int ce = 16 / elem_bytes(y_dtype);
-  const int qb = code_entries == 16 ? ce / 2 : ce;
-  p.vec = aligned(y, 16) && aligned(q, qb);
-  p.nchunks = p.vec ? n / ce : 0;
-  switch (y_dtype) {
-    case BQ_F32: return dispatch_dequant<bq::kF32>(p, code_entries, dev, info.sms, stream);
-    case BQ_F16: return dispatch_dequant<bq::kF16>(p, code_entries, dev, info.sms, stream);
-    default: return dispatch_dequant<bq::kBF16>(p, code_entries, dev, info.sms, stream);
+  return dequant_entry<false>(p, n, blocksize, code_entries, y_dtype, stream);
+}
+
+bq_status bq_quantize_blockwise_nested(const void* x, bq_dtype x_dtype, int64_t n,
+                                       int32_t blocksize, const float* code,
+                                       int32_t code_entries, const float* code2,
+                                       int32_t code2_entries, int32_t blocksize2, float* absmax,
+                                       uint8_t* out, float* absmax2, uint8_t* qabsmax,
+                                       cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(x_dtype) || !valid_blocksize(blocksize) ||
+      !valid_blocksize(blocksize2) || (code_entries != 16 && code_entries != 256) ||
+      code2_entries != 256)
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (!code2 || !absmax2 || !qabsmax || !aligned(code2, 4) || !aligned(absmax2, 4))
+    return BQ_ERR_INVALID_ARG;
+  // the elements, then their fp32 statistics as a second blockwise input
+  bq_status s = bq_quantize_blockwise(x, x_dtype, n, blocksize, code, code_entries, absmax, out,
+                                      stream);
+  if (s != BQ_OK) return s;
+  const int64_t nb = (n + blocksize - 1) / blocksize;
+  return bq_quantize_blockwise(absmax, BQ_F32, nb, blocksize2, code2, code2_entries, absmax2,
+                               qabsmax, stream);
+}
+
+bq_status bq_dequantize_blockwise_nested(const uint8_t* q, const uint8_t* qabsmax,
+                                         const float* absmax2, int64_t n, int32_t blocksize,
+                                         const float* code, int32_t code_entries,
+                                         const float* code2, int32_t code2_entries,
+                                         int32_t blocksize2, void* y, bq_dtype y_dtype,
+                                         cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(y_dtype) || !valid_blocksize(blocksize) ||
+      !valid_blocksize(blocksize2) || (code_entries != 16 && code_entries != 256) ||
+      code2_entries != 256)
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (n > (int64_t{1} << 50)) return BQ_ERR_INVALID_ARG;
+  if (!q || !qabsmax || !absmax2 || !code || !code2 || !y || !aligned(absmax2, 4) ||
+      !aligned(code, 4) || !aligned(code2, 4) || !aligned(y, elem_bytes(y_dtype)))
+    return BQ_ERR_INVALID_ARG;
+  bq::DParams p{};
+  p.q = q;
+  p.code = code;
+  p.y = y;
+  p.qa = qabsmax;
+  p.absmax2 = absmax2;
+  p.code2 = code2;
+  p.bs2_log2 = log2i(blocksize2);
+  return dequant_entry<true>(p, n, blocksize, code_entries, y_dtype, stream);
+}
+
+bq_status bq_quantize_blockwise_host(const void* x_host, bq_dtype x_dtype, int64_t n,
+                                     int32_t blocksize, const float* code, int32_t code_entries,
+                                     const float* code2, int32_t code2_entries,
+                                     int32_t blocksize2, float* absmax, uint8_t* out,
+                                     float* absmax2, uint8_t* qabsmax, void* staging,
+                                     int64_t staging_bytes, int64_t chunk_elements,
+                                     cudaStream_t stream0, cudaStream_t stream1) {
+  t_err.clear();
+  const bool nested = code2 != nullptr;
+  if (n < 0 || !valid_dtype(x_dtype) || !valid_blocksize(blocksize) ||
+      (code_entries != 16 && code_entries != 256))
+    return BQ_ERR_INVALID_ARG;
+  if (nested && (!valid_blocksize(blocksize2) || code2_entries != 256 || !absmax2 || !qabsmax))
+    return BQ_ERR_INVALID_ARG;
+  // chunks are whole blocks (whole second-level blocks with compressed
+  // statistics), so every chunk's outputs start where the whole call's would
+  const int64_t unit = nested ? int64_t{blocksize} * blocksize2 : blocksize;
+  if (chunk_elements <= 0 || chunk_elements % unit != 0 || chunk_elements > (int64_t{1} << 40))
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  const int eb = elem_bytes(x_dtype);
+  const int64_t chunks = (n + chunk_elements - 1) / chunk_elements;
+  const int64_t chunk_bytes = chunk_elements * eb;
+  const int64_t need = chunks > 1 ? 2 * chunk_bytes : n * eb;
+  if (!x_host || !aligned(x_host, eb) || !staging || !aligned(staging, 16) ||
+      staging_bytes < need || !absmax || !out)
+    return BQ_ERR_INVALID_ARG;
+
+  cudaEvent_t joined = nullptr;
+  const bool two = chunks > 1 && stream1 != stream0;
+  if (two) {
+    cudaError_t e = cudaEventCreateWithFlags(&joined, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "pipeline event");
   }
+  bq_status st = BQ_OK;
+  for (int64_t i = 0; i < chunks && st == BQ_OK; ++i) {
+    // chunk i goes to staging half i % 2 on stream i % 2: the copy of one
+    // chunk overlaps the quantization of the other, and a half is refilled
+    // only after the quantization that read it (same stream)
+    const int64_t off = i * chunk_elements;
+    const int64_t len = n - off < chunk_elements ? n - off : chunk_elements;
+    cudaStream_t s = (i & 1) ? stream1 : stream0;
+    void* dst = static_cast<uint8_t*>(staging) + (i & 1) * chunk_bytes;
+    cudaError_t e = cudaMemcpyAsync(dst, static_cast<const uint8_t*>(x_host) + off * eb,
+                                    static_cast<size_t>(len * eb), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "pipeline host-to-device copy");
+      break;
+    }
+    const int64_t b0 = off / blocksize;
+    uint8_t* o = out + (code_entries == 16 ? off / 2 : off);
+    st = nested ? bq_quantize_blockwise_nested(dst, x_dtype, len, blocksize, code, code_entries,
+                                               code2, code2_entries, blocksize2, absmax + b0, o,
+                                               absmax2 + b0 / blocksize2, qabsmax + b0, s)
+                : bq_quantize_blockwise(dst, x_dtype, len, blocksize, code, code_entries,
+                                        absmax + b0, o, s);
+  }
+  if (two) {
+    // stream0 continues only after stream1's chunks
+    cudaError_t e = cudaEventRecord(joined, stream1);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream0, joined, 0);
+    if (e != cudaSuccess && st == BQ_OK) st = cuda_fail(e, "pipeline join");
+    cudaEventDestroy(joined);  // released once the recorded work completes
+  }
+  return st;
 }
 
 bq_status bq_dequant_q8_0(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,

@@ -19,6 +19,13 @@
 // fp32x2 multiply per two elements.  8-bit codes: one 32-bit load per element,
 // multiplied in pairs.  Buffers that are not aligned for the vector path, and
 // the elements after the last whole chunk, are done one element per thread.
+//
+// Compressed statistics ("bitsandbytes PR #2052", Summary: the absmax array of
+// NF4 storage is itself quantized blockwise with the General8 map): with
+// NESTED, block b's scale is rebuilt in the kernel as
+// A_b = RN(code2[qa[b]] * absmax2[b / blocksize2]) - the value the
+// statistics' own dequantization would have stored - from a 256-entry shared
+// table, so no fp32 absmax array is written or read.
 #pragma once
 
 #include "bq_search.cuh"
@@ -27,13 +34,18 @@ namespace bq {
 
 struct DParams {
   const uint8_t* q;
-  const float* absmax;
+  const float* absmax;   // plain statistics
   const float* code;
   void* y;
   int64_t n;
   int64_t nchunks;   // whole 16-byte output chunks taken by the vector path
   int32_t bs_log2;
   int32_t vec;
+  // compressed statistics (NESTED kernels only)
+  const uint8_t* qa;       // one code of code2 per block
+  const float* absmax2;    // one scale per blocksize2 blocks
+  const float* code2;      // 256 entries
+  int32_t bs2_log2;
 };
 
 constexpr int kDThreads = 256;
@@ -46,12 +58,25 @@ struct DTraits {
   static constexpr int QB = E == 16 ? CE / 2 : CE;    // code bytes per chunk
 };
 
-template <int E>
+template <int E, bool NESTED>
 struct DSmem {
   // E == 16: pair[b] = (code[b >> 4], code[b & 15]); E == 256: code[b]
   float t[E == 16 ? 512 : 256];
   float code[E];
+  float code2[NESTED ? 256 : 1];
 };
+
+// Scale of quantization block b: stored, or rebuilt from its code and the
+// second-level scale.
+template <bool NESTED, int E>
+__device__ __forceinline__ float block_scale(const DParams& p, const DSmem<E, NESTED>& s,
+                                             int64_t b) {
+  if constexpr (NESTED) {
+    return __fmul_rn(s.code2[__ldg(p.qa + b)], __ldg(p.absmax2 + (b >> p.bs2_log2)));
+  } else {
+    return __ldg(p.absmax + b);
+  }
+}
 
 template <int QB>
 __device__ __forceinline__ uint2 load_codes(const uint8_t* __restrict__ q, int64_t chunk) {
@@ -104,12 +129,14 @@ __device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, uint32_t t_base)
   }
 }
 
-template <int E, int OT>
+template <int E, int OT, bool NESTED>
 __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
-  __shared__ DSmem<E> s;
+  __shared__ DSmem<E, NESTED> s;
   pdl_release();
   pdl_wait();  // codes, absmax, codebook and y may belong to the previous kernel
   for (int i = threadIdx.x; i < E; i += blockDim.x) s.code[i] = p.code[i];
+  if constexpr (NESTED)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s.code2[i] = p.code2[i];
   __syncthreads();
   if constexpr (E == 16) {
     for (int b = threadIdx.x; b < 256; b += blockDim.x) {
@@ -132,18 +159,28 @@ __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
     for (int64_t base = gtid; base < p.nchunks; base += U * gsz) {
       uint2 c[U];
       float A[U];
+      uint32_t qa[U];  // NESTED: the block's statistics code, looked up after the loads
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t ch = base + u * gsz;
         if (ch < p.nchunks) {
           c[u] = load_codes<T::QB>(p.q, ch);
-          A[u] = __ldg(p.absmax + ((ch * T::CE) >> p.bs_log2));
+          const int64_t b = (ch * T::CE) >> p.bs_log2;
+          if constexpr (NESTED) {
+            qa[u] = __ldg(p.qa + b);
+            A[u] = __ldg(p.absmax2 + (b >> p.bs2_log2));
+          } else {
+            A[u] = __ldg(p.absmax + b);
+          }
         }
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t ch = base + u * gsz;
-        if (ch < p.nchunks) y4[ch] = decode_chunk<E, OT>(c[u], A[u], t_base);
+        if (ch < p.nchunks) {
+          if constexpr (NESTED) A[u] = __fmul_rn(s.code2[qa[u]], A[u]);
+          y4[ch] = decode_chunk<E, OT>(c[u], A[u], t_base);
+        }
       }
     }
   }
@@ -157,7 +194,7 @@ __global__ void __launch_bounds__(kDThreads) dequant_kernel(const DParams p) {
     } else {
       idx = p.q[i];
     }
-    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], p.absmax[i >> p.bs_log2]));
+    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], block_scale<NESTED>(p, s, i >> p.bs_log2)));
   }
 }
 

@@ -104,6 +104,82 @@ BQ_API bq_status bq_dequantize_blockwise(const uint8_t *q, const float *absmax,
                                   cudaStream_t stream);
 
 /*
+ * Blockwise quantization with compressed statistics ("bitsandbytes PR #2052",
+ * Summary: NF4 storage whose absmax array is itself quantized blockwise with
+ * the General8 map).  Two launches on `stream`: the elements as in
+ * bq_quantize_blockwise, writing their fp32 statistics to `absmax`, then that
+ * array as an fp32 input of nb = ceil(n / blocksize) elements, quantized with
+ * `code2` in blocks of `blocksize2`.  No mean is subtracted from the
+ * statistics (the page describes none).
+ *   code2      device, 256 fp32 entries (the General8 map); code2_entries
+ *              must be 256.
+ *   blocksize2 power of two in [32, 4096] (256 is the usual choice).
+ *   absmax     device, nb fp32, written (the first-level statistics).
+ *   absmax2    device, ceil(nb / blocksize2) fp32, written.
+ *   qabsmax    device, nb bytes, written (one code2 index per block).
+ * Other arguments and errors as bq_quantize_blockwise.
+ */
+BQ_API bq_status bq_quantize_blockwise_nested(const void *x, bq_dtype x_dtype, int64_t n,
+                                  int32_t blocksize, const float *code,
+                                  int32_t code_entries, const float *code2,
+                                  int32_t code2_entries, int32_t blocksize2,
+                                  float *absmax, uint8_t *out, float *absmax2,
+                                  uint8_t *qabsmax, cudaStream_t stream);
+
+/*
+ * Inverse of bq_quantize_blockwise_nested, in one launch: block b's scale is
+ * rebuilt as A_b = RN(code2[qabsmax[b]] * absmax2[b / blocksize2]) - exactly
+ * the fp32 value the statistics' own dequantization gives - and then
+ * y_i = narrow_to(y_dtype, RN(code[idx_i] * A_(i / blocksize))).  No fp32
+ * statistics array is needed.
+ */
+BQ_API bq_status bq_dequantize_blockwise_nested(const uint8_t *q, const uint8_t *qabsmax,
+                                  const float *absmax2, int64_t n, int32_t blocksize,
+                                  const float *code, int32_t code_entries,
+                                  const float *code2, int32_t code2_entries,
+                                  int32_t blocksize2, void *y, bq_dtype y_dtype,
+                                  cudaStream_t stream);
+
+/*
+ * Quantization of a HOST input, pipelined over two streams ("bitsandbytes PR
+ * #2052", B300 measurement: the two-stream pinned host-to-device plus
+ * compressed-NF4 pipeline, where each copy and the quantizer that reads it
+ * are chained on one stream).  The input is cut into chunks of
+ * chunk_elements; chunk i is copied into half (i % 2) of `staging` with
+ * cudaMemcpyAsync on stream (i % 2 ? stream1 : stream0) and quantized right
+ * after its copy on the same stream (with compressed statistics when code2 is
+ * not NULL), so one chunk's copy overlaps the other's quantization.  The
+ * outputs are bit-identical to one bq_quantize_blockwise(_nested) call on the
+ * whole input.  At return, stream0 has been made to wait for stream1's work:
+ * the outputs are complete in stream0's order.
+ * Exception to the common contract: this call reads host memory and creates
+ * (and releases) one CUDA event per call.
+ *   x_host        host, n elements of x_dtype.  Pinned (page-locked) memory
+ *                 gives the overlap; pageable memory works but the copies
+ *                 then serialize with the host.  Must stay unchanged until
+ *                 stream0's work completes.
+ *   code2 ...     NULL for plain statistics (code2_entries, blocksize2,
+ *                 absmax2 and qabsmax are then ignored); otherwise as
+ *                 bq_quantize_blockwise_nested.
+ *   absmax, out   device outputs as bq_quantize_blockwise.
+ *   staging       device, 16-byte aligned, staging_bytes >= 2 * chunk_elements
+ *                 * element bytes (n * element bytes when n <= chunk_elements).
+ *   chunk_elements > 0, a multiple of blocksize (of blocksize * blocksize2
+ *                 with compressed statistics).
+ *   stream0, stream1  the two streams (may be equal: no overlap then).
+ * BQ_ERR_INVALID_ARG for bad sizes, pointers or a staging buffer that is too
+ * small; BQ_ERR_CUDA if a copy, launch or the join fails.
+ */
+BQ_API bq_status bq_quantize_blockwise_host(const void *x_host, bq_dtype x_dtype, int64_t n,
+                                  int32_t blocksize, const float *code,
+                                  int32_t code_entries, const float *code2,
+                                  int32_t code2_entries, int32_t blocksize2,
+                                  float *absmax, uint8_t *out, float *absmax2,
+                                  uint8_t *qabsmax, void *staging, int64_t staging_bytes,
+                                  int64_t chunk_elements, cudaStream_t stream0,
+                                  cudaStream_t stream1);
+
+/*
  * GGUF Q8_0 dequantization ("ComfyUI-GGUF PR #472, Cache device-side
  * constants in dequant kernels", Verification table, Q8_0 row: the one type
  * with no shift constant).  Block k is 34 bytes: fp16 d (little endian, bytes

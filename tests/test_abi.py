@@ -27,13 +27,15 @@ def test_header_declares_the_compute_calls():
     syms = declared_symbols()
     for name in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
                  "bq_dequant_q4_0", "bq_dequant_q4_1", "bq_dequant_q5_0", "bq_dequant_q5_1",
-                 "bq_dequant_q4_k", "bq_dequant_q6_k", "bq_quantize_q8_0", "bq_quantize_q4_0"):
+                 "bq_dequant_q4_k", "bq_dequant_q6_k", "bq_quantize_q8_0", "bq_quantize_q4_0",
+                 "bq_quantize_blockwise_nested", "bq_dequantize_blockwise_nested",
+                 "bq_quantize_blockwise_host"):
         assert name in syms
 
 
 def test_every_declared_symbol_is_exported(L):
     syms = declared_symbols()
-    assert len(syms) >= 15
+    assert len(syms) >= 18
     assert set(syms) == set(bq.EXPORTED)
     for name in syms:
         assert hasattr(L, name), name
@@ -100,6 +102,42 @@ def test_rejects_bad_sizes_pointers_dtypes(L):
         assert fn(P + 2, bq.BQ_F32, 64, P, 0) == E, kind
         assert fn(P, 5, 64, P, 0) == E, kind
         assert fn(P, bq.BQ_F32, 1 << 51, P, 0) == E, kind
+
+
+def test_nested_and_host_pipeline_reject_bad_arguments(L):
+    E = bq.BQ_ERR_INVALID_ARG
+    B = bq.BQ_BF16
+    q_n = bq.bq_quantize_blockwise_nested
+    assert q_n(P, B, 4096, 64, P, 16, P, 16, 256, P, P, P, P, 0) == E      # code2 not 256 entries
+    assert q_n(P, B, 4096, 64, P, 16, P, 256, 100, P, P, P, P, 0) == E     # blocksize2
+    assert q_n(P, B, 4096, 64, P, 16, P, 256, 8192, P, P, P, P, 0) == E
+    assert q_n(P, B, 4096, 64, P, 16, 0, 256, 256, P, P, P, P, 0) == E     # null code2
+    assert q_n(P, B, 4096, 64, P, 16, P, 256, 256, P, P, 0, P, 0) == E     # null absmax2
+    assert q_n(P, B, 4096, 64, P, 16, P, 256, 256, P, P, P, 0, 0) == E     # null qabsmax
+    assert q_n(P, B, 4096, 64, P, 16, P + 2, 256, 256, P, P, P, P, 0) == E
+    d_n = bq.bq_dequantize_blockwise_nested
+    assert d_n(P, P, P, 4096, 64, P, 16, P, 16, 256, P, B, 0) == E
+    assert d_n(P, P, P, 4096, 64, P, 16, P, 256, 48, P, B, 0) == E
+    assert d_n(P, 0, P, 4096, 64, P, 16, P, 256, 256, P, B, 0) == E
+    assert d_n(P, P, 0, 4096, 64, P, 16, P, 256, 256, P, B, 0) == E
+    assert d_n(P, P, P, 4096, 64, P, 16, P, 256, 256, P + 1, B, 0) == E
+    assert d_n(P, P, P, -1, 64, P, 16, P, 256, 256, P, B, 0) == E
+    h = bq.bq_quantize_blockwise_host
+    # chunk not whole blocks / not whole second-level blocks / not positive
+    assert h(P, B, 4096, 64, P, 16, None, 0, 0, P, P, None, None, P, 1 << 20, 100, 0, 0) == E
+    assert h(P, B, 4096, 64, P, 16, P, 256, 256, P, P, P, P, P, 1 << 20, 64 * 100, 0, 0) == E
+    assert h(P, B, 4096, 64, P, 16, None, 0, 0, P, P, None, None, P, 1 << 20, 0, 0, 0) == E
+    # staging too small for two chunks, or misaligned
+    assert h(P, B, 1 << 20, 64, P, 16, None, 0, 0, P, P, None, None, P, 4096, 4096, 0, 0) == E
+    assert h(P, B, 4096, 64, P, 16, None, 0, 0, P, P, None, None, P + 8, 1 << 20, 64, 0, 0) == E
+    # null host input, misaligned host input, null outputs
+    assert h(0, B, 4096, 64, P, 16, None, 0, 0, P, P, None, None, P, 1 << 20, 64, 0, 0) == E
+    assert h(P + 1, B, 4096, 64, P, 16, None, 0, 0, P, P, None, None, P, 1 << 20, 64, 0, 0) == E
+    assert h(P, B, 4096, 64, P, 16, None, 0, 0, 0, P, None, None, P, 1 << 20, 64, 0, 0) == E
+    # nested without its outputs
+    assert h(P, B, 4096, 64, P, 16, P, 256, 256, P, P, None, P, P, 1 << 20, 64 * 256, 0, 0) == E
+    # n == 0 is fine with no buffers at all
+    assert h(0, B, 0, 64, 0, 16, None, 0, 0, 0, 0, None, None, 0, 0, 64, 0, 0) == bq.BQ_OK
 
 
 def test_zero_length_is_ok_without_touching_the_device(L):

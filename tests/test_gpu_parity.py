@@ -498,25 +498,141 @@ def test_bounded_wait_gives_up_and_context_survives(probes):
 
 # ------------------------------------------------- compressed statistics ---
 
-@pytest.mark.parametrize("dtype,bs", [("bf16", 64), ("f16", 4096), ("f32", 32)])
-def test_nested_statistics_parity(dtype, bs):
+def _oracle_nested(xh, dtype, bs, bs2, n, ydtype, table=None):
+    """The composition of oracle calls that defines compressed statistics."""
+    nf4, dyn = table if table is not None else TABLES["nf4"], TABLES["dyn8"]
+    oa, oq = oracle.quantize_blockwise(xh, dtype, bs, nf4)
+    oa2, oqa = oracle.quantize_blockwise(oa, "f32", bs2, dyn)
+    oa_back = oracle.dequantize_blockwise(oqa, oa2, oa.size, bs2, dyn, "f32")
+    oy = oracle.dequantize_blockwise(oq, oa_back, n, bs, nf4, ydtype)
+    return oa, oq, oa2, oqa, oy
+
+
+@pytest.mark.parametrize("dtype,bs,bs2", [("bf16", 64, 256), ("f16", 4096, 256), ("f32", 32, 256),
+                                          ("bf16", 256, 32), ("f16", 32, 4096)])
+def test_nested_statistics_parity(dtype, bs, bs2):
     """Compressed statistics: the absmax array quantized with the dynamic
-    8-bit table in blocks of 256, against the same composition of oracle
-    calls."""
+    8-bit table in blocks of blocksize2, against the same composition of
+    oracle calls; the fused dequantization against the oracle's two-step
+    inverse, to every output dtype."""
     n = 300 * bs + 37
-    x = synth.with_zero_block(synth.normal(n, dtype, seed=bs + 1), bs)
+    x = synth.with_zero_block(synth.normal(n, dtype, seed=bs + bs2), bs)
     nf4, dyn = TABLES["nf4"], TABLES["dyn8"]
-    q, qa, a2, a = bq.quantize_blockwise_nested(x.cuda(), code_dev(nf4), bs, code_dev(dyn))
-    y = bq.dequantize_blockwise_nested(q, qa, a2, n, bs, code_dev(nf4), code_dev(dyn),
-                                       dtype=x.dtype)
+    q, qa, a2, a = bq.quantize_blockwise_nested(x.cuda(), code_dev(nf4), bs, code_dev(dyn), bs2)
     torch.cuda.synchronize()
     xh = np_bits(x)
-    oa, oq = oracle.quantize_blockwise(xh, dtype, bs, nf4)
-    oa2, oqa = oracle.quantize_blockwise(oa, "f32", 256, dyn)
-    oa_back = oracle.dequantize_blockwise(oqa, oa2, oa.size, 256, dyn, "f32")
-    oy = oracle.dequantize_blockwise(oq, oa_back, n, bs, nf4, dtype)
+    oa, oq, oa2, oqa, oy = _oracle_nested(xh, dtype, bs, bs2, n, dtype)
     assert np.array_equal(a.cpu().numpy(), oa)
     assert np.array_equal(q.cpu().numpy(), oq)
     assert np.array_equal(qa.cpu().numpy(), oqa)
     assert np.array_equal(a2.cpu().numpy(), oa2)
-    assert np.array_equal(np_bits(y.cpu()), oy)
+    for ydt in ("bf16", "f16", "f32"):
+        y = bq.dequantize_blockwise_nested(q, qa, a2, n, bs, code_dev(nf4), code_dev(dyn), bs2,
+                                           dtype=synth.TORCH_DTYPES[ydt])
+        want = oracle.dequantize_blockwise(
+            oq, oracle.dequantize_blockwise(oqa, oa2, oa.size, bs2, dyn, "f32"), n, bs, nf4, ydt)
+        assert np.array_equal(np_bits(y.cpu()), want), ydt
+    assert bq.bq_device_fault() == 0
+
+
+def test_nested_dequant_unaligned_and_8bit():
+    """The fused nested dequantization on its element-wise path (output not
+    16-byte aligned) and with an 8-bit element codebook."""
+    bs, bs2 = 64, 256
+    n = 517 * bs + 9
+    x = synth.normal(n, "bf16", seed=71)
+    dyn = TABLES["dyn8"]
+    for table in (TABLES["nf4"], dyn):
+        q, qa, a2, a = bq.quantize_blockwise_nested(x.cuda(), code_dev(table), bs, code_dev(dyn),
+                                                    bs2)
+        oa, oq, oa2, oqa, oy = _oracle_nested(np_bits(x), "bf16", bs, bs2, n, "bf16", table)
+        assert np.array_equal(q.cpu().numpy(), oq)
+        y = Guarded(2 * n, offset=2)
+        assert bq.bq_dequantize_blockwise_nested(
+            q.data_ptr(), qa.data_ptr(), a2.data_ptr(), n, bs, code_dev(table).data_ptr(),
+            table.size, code_dev(dyn).data_ptr(), 256, bs2, y.ptr, bq.BQ_BF16, 0) == bq.BQ_OK
+        torch.cuda.synchronize()
+        assert y.guards_intact()
+        assert np.array_equal(y.host().view(np.uint16), oy)
+
+
+def test_nested_rejects_bad_arguments():
+    E = bq.BQ_ERR_INVALID_ARG
+    x = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+    c16 = code_dev(TABLES["nf4"])
+    c256 = code_dev(TABLES["dyn8"])
+    buf = torch.zeros(8192, dtype=torch.uint8, device="cuda")
+    P = buf.data_ptr()
+    # code2 must have 256 entries; blocksize2 a power of two in [32, 4096]
+    assert bq.bq_quantize_blockwise_nested(x.data_ptr(), bq.BQ_BF16, 4096, 64, c16.data_ptr(), 16,
+                                           c16.data_ptr(), 16, 256, P, P, P, P, 0) == E
+    assert bq.bq_quantize_blockwise_nested(x.data_ptr(), bq.BQ_BF16, 4096, 64, c16.data_ptr(), 16,
+                                           c256.data_ptr(), 256, 100, P, P, P, P, 0) == E
+    assert bq.bq_dequantize_blockwise_nested(P, P, P, 4096, 64, c16.data_ptr(), 16, 0, 256, 256,
+                                             P, bq.BQ_BF16, 0) == E
+    assert bq.bq_device_fault() == 0
+
+
+# ------------------------------------------------------ host-input pipeline --
+
+@pytest.mark.parametrize("nested", [False, True])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_pipeline_matches_device_call(nested, pinned):
+    """The two-stream host pipeline gives the bytes of one call on the whole
+    device-resident input: several chunks and a ragged tail, both halves of
+    the staging buffer reused more than once."""
+    bs, bs2 = 64, 256
+    chunk = bs * bs2 * 3                        # 49152 elements
+    n = chunk * 5 + 1000 * bs + 17              # 5 whole chunks and a partial one
+    x = synth.with_zero_block(synth.normal(n, "bf16", seed=5 + nested), bs)
+    xh = x.pin_memory() if pinned else x
+    nf4, dyn = code_dev(TABLES["nf4"]), code_dev(TABLES["dyn8"])
+    if nested:
+        got = bq.quantize_blockwise_host(xh, nf4, bs, dyn, bs2, chunk_elements=chunk)
+        want = bq.quantize_blockwise_nested(x.cuda(), nf4, bs, dyn, bs2)
+    else:
+        got = bq.quantize_blockwise_host(xh, nf4, bs, chunk_elements=chunk)
+        want = bq.quantize_blockwise(x.cuda(), nf4, bs)
+    torch.cuda.synchronize()
+    assert len(got) == len(want)
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)
+    assert bq.bq_device_fault() == 0
+
+
+def test_host_pipeline_single_stream_and_one_chunk():
+    bs = 256
+    n = 3 * 65536 + 5
+    x = synth.normal(n, "f16", seed=8).pin_memory()
+    nf4 = code_dev(TABLES["nf4"])
+    want_a, want_q = bq.quantize_blockwise(x.cuda(), nf4, bs)
+    a = torch.empty_like(want_a)
+    q = torch.empty_like(want_q)
+    staging = torch.empty(2 * 65536 * 2, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    # both streams the same: sequential chunks
+    assert bq.bq_quantize_blockwise_host(x.data_ptr(), bq.BQ_F16, n, bs, nf4.data_ptr(), 16, None,
+                                         0, 0, a.data_ptr(), q.data_ptr(), None, None,
+                                         staging.data_ptr(), staging.numel(), 65536, s, s) == bq.BQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(a, want_a) and torch.equal(q, want_q)
+    # one chunk covering everything needs only one chunk of staging
+    big = torch.empty(n * 2 + 64, dtype=torch.uint8, device="cuda")
+    a.zero_()
+    q.zero_()
+    assert bq.bq_quantize_blockwise_host(x.data_ptr(), bq.BQ_F16, n, bs, nf4.data_ptr(), 16, None,
+                                         0, 0, a.data_ptr(), q.data_ptr(), None, None,
+                                         big.data_ptr(), big.numel(), 1 << 20, s, s) == bq.BQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(a, want_a) and torch.equal(q, want_q)
+    # staging too small, or a chunk that is not whole blocks
+    E = bq.BQ_ERR_INVALID_ARG
+    assert bq.bq_quantize_blockwise_host(x.data_ptr(), bq.BQ_F16, n, bs, nf4.data_ptr(), 16, None,
+                                         0, 0, a.data_ptr(), q.data_ptr(), None, None,
+                                         staging.data_ptr(), staging.numel() - 16, 65536, s,
+                                         s) == E
+    assert bq.bq_quantize_blockwise_host(x.data_ptr(), bq.BQ_F16, n, bs, nf4.data_ptr(), 16, None,
+                                         0, 0, a.data_ptr(), q.data_ptr(), None, None,
+                                         staging.data_ptr(), staging.numel(), 65536 + 128, s,
+                                         s) == E
+    assert bq.bq_device_fault() == 0
