@@ -92,17 +92,26 @@ GGUF_LAYOUT = {
     "q4_1": (20, ((0, False), (2, True))),
     "q5_0": (22, ((0, False),)),
     "q5_1": (24, ((0, False), (2, True))),
+    "q2_k": (84, ((80, False), (82, False))),
+    "q3_k": (110, ((108, False),)),
     "q4_k": (144, ((0, False), (2, False))),
+    "q5_k": (176, ((0, False), (2, False))),
     "q6_k": (210, ((208, False),)),
 }
 
 
 def gguf_blocks(n_blocks, kind, seed=4):
-    """GGUF blocks of `kind` as a uint8 numpy array [n_blocks, block_bytes].
+    """GGUF blocks of `kind` as a uint8 numpy array [n_blocks, block_bytes]
+    ("bf16": n_blocks single values of 2 bytes, N(0, 0.02)).
 
     Each fp16 field is |N(0,1)| * 0.01 (a signed N(0,1) * 0.01 for a min
     field), stored little-endian at its offset; every other byte (quant bytes,
     high-bit words, packed sub-block scales) is uniform on 0..255."""
+    if kind == "bf16":
+        # plain bfloat16 weights, N(0, 0.02): [n_blocks, 2] little-endian bytes
+        g = _gen(seed)
+        v = torch.randn(n_blocks, generator=g).mul_(0.02).to(torch.bfloat16)
+        return v.view(torch.int16).numpy().view(np.uint8).reshape(n_blocks, 2).copy()
     bb, fields = GGUF_LAYOUT[kind]
     g = _gen(seed)
     vals = []

@@ -22,7 +22,8 @@ DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
 
 # GGUF block types: (elements per block, bytes per block)
 GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32, 22),
-              "q5_1": (32, 24), "q4_k": (256, 144), "q6_k": (256, 210)}
+              "q5_1": (32, 24), "q2_k": (256, 84), "q3_k": (256, 110), "q4_k": (256, 144),
+              "q5_k": (256, 176), "q6_k": (256, 210), "bf16": (1, 2)}
 _ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
 
 _lib = None

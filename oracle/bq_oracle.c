@@ -355,6 +355,102 @@ int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
     return 0;
 }
 
+/* Q2_K: sub-block j covers outputs 16j .. 16j + 15.  In half n (outputs
+ * 128n ..), output 32c + 16h + l (c < 4, h < 2, l < 16) takes bits 2c, 2c+1
+ * of qs[32n + 16h + l]; its sub-block is 8n + 2c + h. */
+int bqo_dequant_q2_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 84 * k;
+        const uint8_t *scales = blk, *qs = blk + 16;
+        float d = half_at(blk + 80), dmin = half_at(blk + 82);
+        for (int n = 0; n < 2; ++n)
+            for (int c = 0; c < 4; ++c)
+                for (int h = 0; h < 2; ++h) {
+                    int j = 8 * n + 2 * c + h;
+                    float a = d * (float)(scales[j] & 15), b = dmin * (float)(scales[j] >> 4);
+                    for (int l = 0; l < 16; ++l) {
+                        int q = (qs[32 * n + 16 * h + l] >> (2 * c)) & 3;
+                        store_elem(y, ydtype, 256 * k + 128 * n + 32 * c + 16 * h + l,
+                                   a * (float)q - b);
+                    }
+                }
+    }
+    return 0;
+}
+
+/* Q3_K scale of sub-block i (0..15) from the 12 packed bytes: low 4 bits
+ * from byte i (i < 8) or the high nibble of byte i - 8, top 2 bits from
+ * byte 8 + i % 4 at bit 2 * (i / 4); stored with an offset of 32. */
+static int q3k_scale(const uint8_t *sc, int i)
+{
+    int lo = i < 8 ? (sc[i] & 15) : (sc[i - 8] >> 4);
+    int hi = (sc[8 + (i & 3)] >> (2 * (i >> 2))) & 3;
+    return (lo | (hi << 4)) - 32;
+}
+
+/* Q3_K: output 128n + 32c + 16h + l takes bits 2c, 2c+1 of qs[32n + 16h + l]
+ * and bit 4n + c of hmask[16h + l]; q = low bits - (hmask bit ? 0 : 4). */
+int bqo_dequant_q3_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 110 * k;
+        const uint8_t *hmask = blk, *qs = blk + 32, *scales = blk + 96;
+        float d = half_at(blk + 108);
+        for (int n = 0; n < 2; ++n)
+            for (int c = 0; c < 4; ++c)
+                for (int h = 0; h < 2; ++h) {
+                    float a = d * (float)q3k_scale(scales, 8 * n + 2 * c + h);
+                    for (int l = 0; l < 16; ++l) {
+                        int low = (qs[32 * n + 16 * h + l] >> (2 * c)) & 3;
+                        int hb = (hmask[16 * h + l] >> (4 * n + c)) & 1;
+                        int q = low - (hb ? 0 : 4);
+                        store_elem(y, ydtype, 256 * k + 128 * n + 32 * c + 16 * h + l,
+                                   a * (float)q);
+                    }
+                }
+    }
+    return 0;
+}
+
+/* Q5_K: as Q4_K (group g of 64 reads qs[32g ..], low nibbles for sub-block
+ * 2g, high for 2g + 1) plus bit 2g + h of qh[l] as bit 4 of q. */
+int bqo_dequant_q5_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype)
+{
+    if (n_blocks < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t k = 0; k < n_blocks; ++k) {
+        const uint8_t *blk = blocks + 176 * k;
+        float d = half_at(blk), dmin = half_at(blk + 2);
+        const uint8_t *scales = blk + 4, *qh = blk + 16, *qs = blk + 48;
+        for (int g = 0; g < 4; ++g)
+            for (int h = 0; h < 2; ++h) {
+                int sci, mni;
+                q4k_scale_min(scales, 2 * g + h, &sci, &mni);
+                float a = d * (float)sci, b = dmin * (float)mni;
+                for (int l = 0; l < 32; ++l) {
+                    int nib = h ? (qs[32 * g + l] >> 4) : (qs[32 * g + l] & 15);
+                    int q = nib | (((qh[l] >> (2 * g + h)) & 1) << 4);
+                    store_elem(y, ydtype, 256 * k + 64 * g + 32 * h + l, a * (float)q - b);
+                }
+            }
+    }
+    return 0;
+}
+
+int bqo_dequant_bf16(const uint8_t *src, int64_t n, void *y, int ydtype)
+{
+    if (n < 0 || !valid_dtype(ydtype))
+        return -1;
+    for (int64_t i = 0; i < n; ++i)
+        store_elem(y, ydtype, i, bqo_bf16_to_f32((uint16_t)(src[2 * i] | (src[2 * i + 1] << 8))));
+    return 0;
+}
+
 /* ------------------------------------------------------- GGUF encoders -- */
 
 static void put_half(uint8_t *p, float v)

@@ -1,7 +1,7 @@
 /*
  * bq_oracle.h - plain, slow, single-threaded CPU reference for blockwise
  * codebook quantization / dequantization and GGUF block dequantization
- * (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K).
+ * (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q2_K, Q3_K, Q4_K, Q5_K, Q6_K, BF16).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the library path may include, link
  * or call this code: only the tests, the package's smoke check and the
@@ -16,8 +16,9 @@
  *  - "ComfyUI-GGUF PR #472, Cache device-side constants in dequant kernels",
  *    Problem section (Q4_0 low nibble then high nibble, shift vector [0, 4])
  *    and the Verification table (Q8_0 and Q4_0 rows).
- *  - The same page's Verification table also lists Q4_1, Q5_0, Q5_1, Q4_K
- *    and Q6_K (4096 blocks, bf16 target, bit-identical).  The pages do not
+ *  - The same page's Verification table also lists Q4_1, Q5_0, Q5_1, Q2_K,
+ *    Q3_K, Q4_K, Q5_K, Q6_K and BF16 (4096 blocks, bf16 target,
+ *    bit-identical).  The pages do not
  *    spell out those block layouts; the functions below follow the GGUF
  *    format's published block layouts, and the tests pin them against the
  *    gguf package's own dequantizer and hand-worked blocks.
@@ -95,6 +96,26 @@ int bqo_dequant_q4_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtyp
  * int8 scales[16], fp16 d}: 16 sub-blocks of 16, y = d*scale*(q - 32) with q
  * the 6-bit value (4 low bits from ql, 2 high bits from qh). */
 int bqo_dequant_q6_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q2_K: 84-byte super-blocks of 256 {uint8 scales[16], uint8 qs[64],
+ * fp16 d, fp16 dmin}: 16 sub-blocks of 16, scale byte j = (min << 4) | scale;
+ * y = d*scale*q - dmin*min with q the 2-bit value. */
+int bqo_dequant_q2_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q3_K: 110-byte super-blocks of 256 {uint8 hmask[32], uint8 qs[64],
+ * uint8 scales[12], fp16 d}: 16 sub-blocks of 16 with 6-bit scales s
+ * (value s - 32); q = 2 low bits from qs, minus 4 when the hmask bit is 0;
+ * y = d*(s - 32)*q. */
+int bqo_dequant_q3_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF Q5_K: 176-byte super-blocks of 256 {fp16 d, fp16 dmin, uint8
+ * scales[12] (packed as Q4_K), uint8 qh[32], uint8 qs[128]}: as Q4_K with a
+ * fifth bit from qh; y = d*sc*q - dmin*mn. */
+int bqo_dequant_q5_k(const uint8_t *blocks, int64_t n_blocks, void *y, int ydtype);
+
+/* GGUF BF16: n raw bfloat16 values (little endian) widened exactly, then
+ * narrowed to ydtype. */
+int bqo_dequant_bf16(const uint8_t *src, int64_t n, void *y, int ydtype);
 
 /*
  * GGUF encoders (the inverse direction of Q8_0 / Q4_0), following the GGUF

@@ -52,6 +52,17 @@ MUTANTS = [
     ("q6k_offset", "int q = (lo4 | (hi2 << 4)) - 32;", "int q = (lo4 | (hi2 << 4)) - 31;"),
     ("q6k_scale_index", "sc[8 * n + l / 16 + 2 * c]", "sc[8 * n + l / 16 + c]"),
     ("q6k_qh_shift", "int hi2 = (qh[32 * n + l] >> (2 * c)) & 3;", "int hi2 = (qh[32 * n + l] >> c) & 3;"),
+    ("q2k_scale_min_swapped",
+     "float a = d * (float)(scales[j] & 15), b = dmin * (float)(scales[j] >> 4);",
+     "float a = d * (float)(scales[j] >> 4), b = dmin * (float)(scales[j] & 15);"),
+    ("q2k_shift", "int q = (qs[32 * n + 16 * h + l] >> (2 * c)) & 3;",
+     "int q = (qs[32 * n + 16 * h + l] >> c) & 3;"),
+    ("q3k_hmask_polarity", "int q = low - (hb ? 0 : 4);", "int q = low - (hb ? 4 : 0);"),
+    ("q3k_top_bits", "int hi = (sc[8 + (i & 3)] >> (2 * (i >> 2))) & 3;",
+     "int hi = (sc[8 + (i >> 2)] >> (2 * (i & 3))) & 3;"),
+    ("q3k_no_offset", "return (lo | (hi << 4)) - 32;", "return (lo | (hi << 4));"),
+    ("q5k_qh_bit", "int q = nib | (((qh[l] >> (2 * g + h)) & 1) << 4);",
+     "int q = nib | (((qh[l] >> (g + h)) & 1) << 4);"),
     ("q8_enc_divisor", "float d = amax / 127.0f;", "float d = amax / 128.0f;"),
     ("q8_enc_round_half_even", "float r = roundf(load_elem(x, dtype, 32 * k + j) * id);",
      "float r = rintf(load_elem(x, dtype, 32 * k + j) * id);"),

@@ -95,11 +95,11 @@ def _load_hand_blocks():
 
 def test_gguf_hand_worked_blocks():
     recs = _load_hand_blocks()
-    assert len(recs) == 12
+    assert len(recs) == 16
     assert {r[0] for r in recs} == set(oracle.GGUF_TYPES)
     for kind, blk, expect in recs:
         per, bb = oracle.GGUF_TYPES[kind]
-        assert blk.size == bb and expect.size == per, kind
+        assert blk.size % bb == 0 and expect.size == per * (blk.size // bb), kind
         fn = lambda b, dt, kind=kind: oracle.dequant_gguf(kind, b, dt)
         y = fn(blk, "f32")
         # bit equality (keeps the sign of zero: d = -0.5 times q = 0 is -0)
@@ -146,10 +146,12 @@ def test_gguf_matches_gguf_package():
     import gguf
     T = gguf.GGMLQuantizationType
     qts = {"q8_0": T.Q8_0, "q4_0": T.Q4_0, "q4_1": T.Q4_1, "q5_0": T.Q5_0, "q5_1": T.Q5_1,
-           "q4_k": T.Q4_K, "q6_k": T.Q6_K}
+           "q2_k": T.Q2_K, "q3_k": T.Q3_K, "q4_k": T.Q4_K, "q5_k": T.Q5_K, "q6_k": T.Q6_K,
+           "bf16": T.BF16}
     assert set(qts) == set(oracle.GGUF_TYPES)
     for kind, qt in qts.items():
-        blocks = synth.gguf_blocks(512 if oracle.GGUF_TYPES[kind][0] == 32 else 64, kind, seed=11)
+        per = oracle.GGUF_TYPES[kind][0]
+        blocks = synth.gguf_blocks({32: 512, 256: 64, 1: 4096}[per], kind, seed=11)
         ref = gq.dequantize(blocks.reshape(-1), qt).astype(np.float32).reshape(-1)
         y = oracle.dequant_gguf(kind, blocks, "f32")
         assert np.array_equal(y.view(np.uint32), ref.view(np.uint32)), kind
