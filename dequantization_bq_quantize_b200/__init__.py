@@ -1,6 +1,7 @@
-"""Blockwise codebook quantization / dequantization and GGUF block
-dequantization (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K) on NVIDIA B200
-(sm_100a).
+"""Blockwise codebook quantization / dequantization (plain and with compressed
+statistics), GGUF block dequantization (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q2_K,
+Q3_K, Q4_K, Q5_K, Q6_K, BF16), GGUF Q8_0 / Q4_0 encoding, and a two-stream
+host-input quantization pipeline, on NVIDIA B200 (sm_100a).
 
 A thin ctypes binding over ``libbq.so`` (C ABI in ``include/bq.h``).  Every
 step of the computation runs in the library's CUDA kernels; this module only
@@ -22,8 +23,10 @@ BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_CUDA = 0, 1, 2, 3
 BQ_F32, BQ_F16, BQ_BF16 = 0, 1, 2
 
 # GGUF block types: (outputs per block, bytes per block)
+# ("bf16": plain bfloat16 values, one per 2-byte "block")
 GGUF_TYPES = {"q8_0": (32, 34), "q4_0": (32, 18), "q4_1": (32, 20), "q5_0": (32, 22),
-              "q5_1": (32, 24), "q4_k": (256, 144), "q6_k": (256, 210)}
+              "q5_1": (32, 24), "q2_k": (256, 84), "q3_k": (256, 110), "q4_k": (256, 144),
+              "q5_k": (256, 176), "q6_k": (256, 210), "bf16": (1, 2)}
 
 GGUF_ENCODERS = ("q8_0", "q4_0")
 
@@ -162,6 +165,22 @@ def bq_quantize_q4_0(x, x_dtype, n, blocks, stream):
     return lib().bq_quantize_q4_0(x, x_dtype, n, blocks, stream)
 
 
+def bq_dequant_q2_k(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q2_k(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q3_k(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q3_k(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_q5_k(blocks, n_blocks, y, y_dtype, stream):
+    return lib().bq_dequant_q5_k(blocks, n_blocks, y, y_dtype, stream)
+
+
+def bq_dequant_bf16(x, n, y, y_dtype, stream):
+    return lib().bq_dequant_bf16(x, n, y, y_dtype, stream)
+
+
 def bq_status_string(status):
     return lib().bq_status_string(status).decode()
 
@@ -296,6 +315,26 @@ def dequant_q5_0(blocks, dtype=None, out=None, stream=None):
 def dequant_q5_1(blocks, dtype=None, out=None, stream=None):
     """GGUF Q5_1 blocks (n_blocks*24 bytes) -> 32*n_blocks values."""
     return dequant_gguf("q5_1", blocks, dtype, out, stream)
+
+
+def dequant_q2_k(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q2_K super-blocks (n_blocks*84 bytes) -> 256*n_blocks values."""
+    return dequant_gguf("q2_k", blocks, dtype, out, stream)
+
+
+def dequant_q3_k(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q3_K super-blocks (n_blocks*110 bytes) -> 256*n_blocks values."""
+    return dequant_gguf("q3_k", blocks, dtype, out, stream)
+
+
+def dequant_q5_k(blocks, dtype=None, out=None, stream=None):
+    """GGUF Q5_K super-blocks (n_blocks*176 bytes) -> 256*n_blocks values."""
+    return dequant_gguf("q5_k", blocks, dtype, out, stream)
+
+
+def dequant_bf16(values, dtype=None, out=None, stream=None):
+    """GGUF BF16 tensor data (uint8 CUDA tensor of 2*n bytes) -> n values."""
+    return dequant_gguf("bf16", values, dtype, out, stream)
 
 
 def dequant_q4_k(blocks, dtype=None, out=None, stream=None):

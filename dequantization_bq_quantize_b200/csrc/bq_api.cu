@@ -266,6 +266,22 @@ bq_status gguf_entry(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_d
   }
 }
 
+template <int OT>
+bq_status launch_bf16(const bq::BParams& p, int dev, int sms, cudaStream_t stream) {
+  static KernelSlot slot;
+  auto kernel = bq::bf16_kernel<OT>;
+  int occ = 1;
+  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kGThreads, 0, &occ);
+  if (s != BQ_OK) return s;
+  const int64_t work = p.ngroups > 0 ? p.ngroups : p.n;
+  int64_t want = (work + bq::kGThreads - 1) / bq::kGThreads;
+  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kGThreads, 0, stream, p);
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "bf16 conversion launch");
+}
+
 template <int KIND, int IT>
 bq_status launch_gguf_encode(const bq::GEParams& p, int dev, int sms, cudaStream_t stream) {
   static KernelSlot slot;
@@ -535,6 +551,44 @@ bq_status bq_dequant_q4_k(const void* blocks, int64_t n_blocks, void* y, bq_dtyp
 bq_status bq_dequant_q6_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
                           cudaStream_t stream) {
   return gguf_entry<bq::kQ6_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q2_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ2_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q3_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ3_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_q5_k(const void* blocks, int64_t n_blocks, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  return gguf_entry<bq::kQ5_K>(blocks, n_blocks, y, y_dtype, stream);
+}
+
+bq_status bq_dequant_bf16(const void* x, int64_t n, void* y, bq_dtype y_dtype,
+                          cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(y_dtype)) return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  if (n > (int64_t{1} << 56)) return BQ_ERR_INVALID_ARG;
+  if (!x || !y || !aligned(x, 2) || !aligned(y, elem_bytes(y_dtype))) return BQ_ERR_INVALID_ARG;
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+  bq::BParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.y = y;
+  p.n = n;
+  p.ngroups = aligned(x, 16) && aligned(y, 16) ? n / 8 : 0;
+  switch (y_dtype) {
+    case BQ_F32: return launch_bf16<bq::kF32>(p, dev, info.sms, stream);
+    case BQ_F16: return launch_bf16<bq::kF16>(p, dev, info.sms, stream);
+    default: return launch_bf16<bq::kBF16>(p, dev, info.sms, stream);
+  }
 }
 
 bq_status bq_quantize_q8_0(const void* x, bq_dtype x_dtype, int64_t n, void* blocks,

@@ -1,5 +1,5 @@
 // bq_gguf.cuh - GGUF block dequantization (sm_100a): Q8_0, Q4_0, Q4_1, Q5_0,
-// Q5_1, Q4_K, Q6_K.
+// Q5_1, Q2_K, Q3_K, Q4_K, Q5_K, Q6_K, and the BF16 conversion.
 //
 // Formats.  Q8_0 and Q4_0 as on "ComfyUI-GGUF PR #472, Cache device-side
 // constants in dequant kernels", Problem section and Verification table:
@@ -15,7 +15,13 @@
 //          scales and mins for 8 sub-blocks of 32, qs[128]:  y = d*sc*q - dmin*mn
 //   Q6_K = super-block of 256: ql[128], qh[64], int8 scales[16], fp16 d:
 //          y = d * sc * (q - 32), q = 4 bits of ql | 2 bits of qh << 4
-// Every product here is exact in fp32 (an 11-bit d times at most 6 + 5 more
+//   Q2_K = super-block of 256: scales[16] (min << 4 | scale), qs[64], fp16 d,
+//          fp16 dmin: y = d*sc*q - dmin*mn, q 2 bits
+//   Q3_K = super-block of 256: hmask[32], qs[64], 12 bytes of packed 6-bit
+//          scales, fp16 d: y = d*(s - 32)*q, q = 2 bits - (hmask bit ? 0 : 4)
+//   Q5_K = super-block of 256: fp16 d, fp16 dmin, scales as Q4_K, qh[32],
+//          qs[128]: y = d*sc*q - dmin*mn, q = nibble | qh bit << 4
+// Every product here is exact in fp32 (an 11-bit d times at most 7 + 5 more
 // bits), so the only rounding before the narrowing is the add of a min,
 // done as one fma: the narrowed output is the correctly rounded value.  The
 // page's point - no per-call host-to-device constants - holds trivially here:
@@ -38,7 +44,10 @@
 
 namespace bq {
 
-enum : int { kQ8_0 = 0, kQ4_0 = 1, kQ4_1 = 2, kQ5_0 = 3, kQ5_1 = 4, kQ4_K = 5, kQ6_K = 6 };
+enum : int {
+  kQ8_0 = 0, kQ4_0 = 1, kQ4_1 = 2, kQ5_0 = 3, kQ5_1 = 4, kQ4_K = 5, kQ6_K = 6,
+  kQ2_K = 7, kQ3_K = 8, kQ5_K = 9
+};
 
 struct GParams {
   const uint8_t* blocks;
@@ -59,6 +68,9 @@ template <> struct GTraits<kQ5_0> { static constexpr int BB = 22, EPB = 32, QS =
 template <> struct GTraits<kQ5_1> { static constexpr int BB = 24, EPB = 32, QS = 8, QH = 4; static constexpr bool MIN = true; };
 template <> struct GTraits<kQ4_K> { static constexpr int BB = 144, EPB = 256, QS = 16, QH = 0; static constexpr bool MIN = true; };
 template <> struct GTraits<kQ6_K> { static constexpr int BB = 210, EPB = 256, QS = 0, QH = 128; static constexpr bool MIN = false; };
+template <> struct GTraits<kQ2_K> { static constexpr int BB = 84, EPB = 256, QS = 16, QH = 0; static constexpr bool MIN = true; };
+template <> struct GTraits<kQ3_K> { static constexpr int BB = 110, EPB = 256, QS = 32, QH = 0; static constexpr bool MIN = false; };
+template <> struct GTraits<kQ5_K> { static constexpr int BB = 176, EPB = 256, QS = 48, QH = 16; static constexpr bool MIN = true; };
 
 // blocks per warp step: 32 blocks of 32 or 8 super-blocks of 256
 template <int KIND> struct GStep { static constexpr int value = GTraits<KIND>::EPB == 32 ? 32 : 8; };
@@ -157,6 +169,48 @@ __device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float 
     w0 = (q.x >> (4 * h)) & 0x0F0F0F0Fu;
     w1 = (q.y >> (4 * h)) & 0x0F0F0F0Fu;
     bytes_to_values<true>(w0, w1, 8388608.0f, a, -b, v);
+  } else if constexpr (KIND == kQ5_K) {
+    // as Q4_K, plus bit 2g + h of qh[8r ..] as bit 4
+    const int g = part >> 3, h = (part >> 2) & 1, r = part & 3;
+    const int is = 2 * g + h, j = is & 3;
+    const uint32_t A = bp[4 + j], B = bp[8 + j], C = bp[12 + j];
+    const bool hi = is >= 4;
+    const uint32_t sc = hi ? ((C & 15u) | ((A >> 6) << 4)) : (A & 63u);
+    const uint32_t mn = hi ? ((C >> 4) | ((B >> 6) << 4)) : (B & 63u);
+    const float a = half_at(bp) * static_cast<float>(sc);        // exact
+    const float b = half_at(bp + 2) * static_cast<float>(mn);    // exact
+    const uint2 q = *reinterpret_cast<const uint2*>(bp + 48 + 32 * g + 8 * r);  // 8-byte aligned
+    const uint2 hb = *reinterpret_cast<const uint2*>(bp + 16 + 8 * r);
+    w0 = ((q.x >> (4 * h)) & 0x0F0F0F0Fu) | (((hb.x >> is) & 0x01010101u) << 4);
+    w1 = ((q.y >> (4 * h)) & 0x0F0F0F0Fu) | (((hb.y >> is) & 0x01010101u) << 4);
+    bytes_to_values<true>(w0, w1, 8388608.0f, a, -b, v);
+  } else if constexpr (KIND == kQ2_K) {
+    // part = 16n + 4c + 2h + s: outputs 128n + 32c + 16h + 8s .., 2-bit field c
+    // of qs[32n + 16h + 8s ..], sub-block part / 2
+    const int n = part >> 4, c = (part >> 2) & 3, hh = (part >> 1) & 1, s8 = (part & 1) * 8;
+    const uint32_t scb = bp[part >> 1];
+    const float a = half_at(bp + 80) * static_cast<float>(scb & 15u);  // exact
+    const float b = half_at(bp + 82) * static_cast<float>(scb >> 4);   // exact
+    load8_at2(bp + 16 + 32 * n + 16 * hh + s8, w0, w1);
+    w0 = (w0 >> (2 * c)) & 0x03030303u;
+    w1 = (w1 >> (2 * c)) & 0x03030303u;
+    bytes_to_values<true>(w0, w1, 8388608.0f, a, -b, v);
+  } else if constexpr (KIND == kQ3_K) {
+    // part = 16n + 4c + 2h + s as Q2_K; bit 4n + c of hmask[16h + 8s ..]
+    // clear means q - 4: the byte (low | hbit << 2) minus 4 is q
+    const int n = part >> 4, c = (part >> 2) & 3, hh = (part >> 1) & 1, s8 = (part & 1) * 8;
+    const int i = part >> 1;  // sub-block
+    const uint32_t lo4 = i < 8 ? (bp[96 + i] & 15u) : (bp[96 + i - 8] >> 4);
+    const uint32_t hi2 = (bp[104 + (i & 3)] >> (2 * (i >> 2))) & 3u;
+    const int scale = static_cast<int>(lo4 | (hi2 << 4)) - 32;
+    const float a = half_at(bp + 108) * static_cast<float>(scale);  // exact
+    uint32_t m0, m1;
+    load8_at2(bp + 32 + 32 * n + 16 * hh + s8, w0, w1);
+    load8_at2(bp + 16 * hh + s8, m0, m1);
+    const int hs = 4 * n + c;
+    w0 = ((w0 >> (2 * c)) & 0x03030303u) | (((m0 >> hs) & 0x01010101u) << 2);
+    w1 = ((w1 >> (2 * c)) & 0x03030303u) | (((m1 >> hs) & 0x01010101u) << 2);
+    bytes_to_values<false>(w0, w1, 8388612.0f /* 2^23 + 4 */, a, 0.0f, v);
   } else {  // kQ6_K
     // part = 16n + 4c + r: half n, 32-element chunk c, outputs 8r..8r+7 of it
     const int n = part >> 4, c = (part >> 2) & 3, r = part & 3;
@@ -258,6 +312,45 @@ __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
       }
     }
     __syncwarp();
+  }
+}
+
+// GGUF BF16 ("ComfyUI-GGUF PR #472", Verification table, BF16 row): plain
+// bfloat16 values, widened exactly and narrowed to the output type (a copy
+// for a bf16 output).  One thread per 8 values (16 bytes in); the elements
+// after the last whole group, and unaligned buffers, one per thread.
+struct BParams {
+  const uint16_t* x;
+  void* y;
+  int64_t n;
+  int64_t ngroups;  // whole groups of 8 taken by the vector path
+};
+
+template <int OT>
+__global__ void __launch_bounds__(kGThreads) bf16_kernel(const BParams p) {
+  pdl_release();
+  pdl_wait();
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t gsz = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t gi = gtid; gi < p.ngroups; gi += gsz) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.x) + gi);
+    if constexpr (OT == kBF16) {
+      reinterpret_cast<uint4*>(p.y)[gi] = w;
+    } else {
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(ws[k] << 16);
+        v[2 * k + 1] = __uint_as_float(ws[k] & 0xffff0000u);
+      }
+      store8<OT>(p.y, gi * 8, v, true);
+    }
+  }
+  for (int64_t i = p.ngroups * 8 + gtid; i < p.n; i += gsz) {
+    const uint32_t h = p.x[i];
+    if constexpr (OT == kBF16) static_cast<uint16_t*>(p.y)[i] = static_cast<uint16_t>(h);
+    else store_elem<OT>(p.y, i, __uint_as_float(h << 16));
   }
 }
 

@@ -1,7 +1,9 @@
 /*
- * bq.h - blockwise codebook quantization / dequantization and GGUF block
- * dequantization (Q8_0, Q4_0, Q4_1, Q5_0, Q5_1, Q4_K, Q6_K) on NVIDIA B200
- * (sm_100a).  C ABI of libbq.so.
+ * bq.h - blockwise codebook quantization / dequantization (plain and with
+ * compressed statistics), GGUF block dequantization (Q8_0, Q4_0, Q4_1, Q5_0,
+ * Q5_1, Q2_K, Q3_K, Q4_K, Q5_K, Q6_K, BF16), GGUF Q8_0 / Q4_0 encoding and a
+ * two-stream host-input quantization pipeline on NVIDIA B200 (sm_100a).
+ * C ABI of libbq.so.
  *
  * Common contract of every compute entry point
  * -------------------------------------------
@@ -205,8 +207,8 @@ BQ_API bq_status bq_dequant_q4_0(const void *blocks, int64_t n_blocks, void *y,
 
 /*
  * The other block types of the same page's Verification table (Q4_1, Q5_0,
- * Q5_1, Q4_K, Q6_K: 4096 blocks, bf16 target, bit-identical across
- * implementations).  The page names them without spelling out their bytes;
+ * Q5_1, Q2_K, Q3_K, Q4_K, Q5_K, Q6_K: 4096 blocks, bf16 target,
+ * bit-identical across implementations; BF16 below).  The page names them without spelling out their bytes;
  * these entry points follow the GGUF block layouts below.  All fp16 fields are
  * little endian; every product is exact in fp32, so the output is the
  * correctly rounded value of the formula, the min being added once.
@@ -256,6 +258,46 @@ BQ_API bq_status bq_dequant_q4_k(const void *blocks, int64_t n_blocks, void *y,
  */
 BQ_API bq_status bq_dequant_q6_k(const void *blocks, int64_t n_blocks, void *y,
                           bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q2_K: 84-byte super-blocks {scales[16], qs[64], fp16 d, fp16 dmin}, 256
+ * outputs in 16 sub-blocks of 16; scales[j] = (min_j << 4) | scale_j.  In
+ * half n (outputs 128n ..), output 32c + 16h + l (c < 4, h < 2, l < 16) takes
+ * bits 2c, 2c + 1 of qs[32n + 16h + l] and belongs to sub-block 8n + 2c + h:
+ *   y = d * scale * q - dmin * min
+ */
+BQ_API bq_status bq_dequant_q2_k(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q3_K: 110-byte super-blocks {hmask[32], qs[64], scales[12], fp16 d}, 16
+ * sub-blocks of 16 with 6-bit scales s_i: the low 4 bits are byte i (i < 8)
+ * or the high nibble of byte i - 8, the top 2 bits come from byte 8 + i % 4
+ * at bit 2 * (i / 4).  Output 128n + 32c + 16h + l takes bits 2c, 2c + 1 of
+ * qs[32n + 16h + l] as q, minus 4 unless bit 4n + c of hmask[16h + l] is set:
+ *   y = d * (s - 32) * q
+ */
+BQ_API bq_status bq_dequant_q3_k(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Q5_K: 176-byte super-blocks {fp16 d, fp16 dmin, scales[12] packed as Q4_K,
+ * qh[32], qs[128]}: as Q4_K, with bit 2g + h of qh[l] (l < 32 the position in
+ * the 32-output half) as bit 4 of q:
+ *   y = d * scale * q - dmin * min
+ */
+BQ_API bq_status bq_dequant_q5_k(const void *blocks, int64_t n_blocks, void *y,
+                          bq_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * BF16 tensor data (the BF16 row of the same table): n little-endian
+ * bfloat16 values widened exactly to fp32 and narrowed to y_dtype (a copy for
+ * BQ_BF16).  x must be 2-byte aligned; n counts values, not blocks.  NaN
+ * payloads are outside the contract (a bf16 output copies them; other
+ * outputs give the conversion's NaN).
+ */
+BQ_API bq_status bq_dequant_bf16(const void *x, int64_t n, void *y, bq_dtype y_dtype,
+                          cudaStream_t stream);
 
 /*
  * GGUF Q8_0 / Q4_0 encoders: the inverse direction of bq_dequant_q8_0 and

@@ -28,6 +28,7 @@ def test_header_declares_the_compute_calls():
     for name in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_dequant_q8_0",
                  "bq_dequant_q4_0", "bq_dequant_q4_1", "bq_dequant_q5_0", "bq_dequant_q5_1",
                  "bq_dequant_q4_k", "bq_dequant_q6_k", "bq_quantize_q8_0", "bq_quantize_q4_0",
+                 "bq_dequant_q2_k", "bq_dequant_q3_k", "bq_dequant_q5_k", "bq_dequant_bf16",
                  "bq_quantize_blockwise_nested", "bq_dequantize_blockwise_nested",
                  "bq_quantize_blockwise_host"):
         assert name in syms
@@ -35,7 +36,7 @@ def test_header_declares_the_compute_calls():
 
 def test_every_declared_symbol_is_exported(L):
     syms = declared_symbols()
-    assert len(syms) >= 18
+    assert len(syms) >= 22
     assert set(syms) == set(bq.EXPORTED)
     for name in syms:
         assert hasattr(L, name), name
@@ -82,6 +83,7 @@ def test_rejects_bad_sizes_pointers_dtypes(L):
     assert bq.bq_dequant_q4_0(0, 10, P, bq.BQ_BF16, 0) == E
     assert bq.bq_dequant_q4_0(P, 10, P + 1, bq.BQ_BF16, 0) == E
     assert bq.bq_dequant_q4_0(P, 10, P, 9, 0) == E
+    assert bq.bq_dequant_bf16(P + 1, 10, P, bq.BQ_F32, 0) == E       # x not 2-byte aligned
     for kind in bq.GGUF_TYPES:
         fn = getattr(bq, "bq_dequant_" + kind)
         assert fn(P, -1, P, bq.BQ_BF16, 0) == E, kind
@@ -90,7 +92,7 @@ def test_rejects_bad_sizes_pointers_dtypes(L):
         assert fn(P, 10, P + 1, bq.BQ_F16, 0) == E, kind
         assert fn(P, 10, P + 2, bq.BQ_F32, 0) == E, kind
         assert fn(P, 10, P, 3, 0) == E, kind
-        assert fn(P, 1 << 53, P, bq.BQ_BF16, 0) == E, kind
+        assert fn(P, 1 << 57, P, bq.BQ_BF16, 0) == E, kind
     for kind in bq.GGUF_ENCODERS:
         fn = getattr(bq, "bq_quantize_" + kind)
         assert fn(P, bq.BQ_BF16, -32, P, 0) == E, kind

@@ -239,8 +239,9 @@ def test_gguf_parity(kind, ydtype):
     single blocks, and streams at byte offsets 1, 2 and 16."""
     per, bb = bq.GGUF_TYPES[kind]
     fn = getattr(bq, "bq_dequant_" + kind)
+    odd = 1 if kind != "bf16" else 2      # bf16 data must be 2-byte aligned
     for nblk, off in ((4096, 0), (4096 * 14336 // per, 0), (1, 0), (7, 0), (8, 0), (9, 0),
-                      (1000 + 3, 0), (1003, 2), (517, 1), (64, 16)):
+                      (1000 + 3, 0), (1003, 2), (517, odd), (64, 16)):
         blocks = synth.gguf_blocks(nblk, kind, seed=4 + nblk)
         bt, bp = device_copy(blocks, off)
         y = Guarded(EB[ydtype] * per * nblk)
@@ -255,11 +256,11 @@ def test_gguf_parity(kind, ydtype):
 def test_gguf_hand_blocks_on_gpu():
     import test_oracle_pins as pins
     for kind, blk, expect in pins._load_hand_blocks():
-        per, _ = bq.GGUF_TYPES[kind]
+        per, bb = bq.GGUF_TYPES[kind]
         fn = getattr(bq, "bq_dequant_" + kind)
         bt, bp = device_copy(blk)
-        y = Guarded(4 * per)
-        assert fn(bp, 1, y.ptr, bq.BQ_F32, 0) == bq.BQ_OK
+        y = Guarded(4 * expect.size)
+        assert fn(bp, blk.size // bb, y.ptr, bq.BQ_F32, 0) == bq.BQ_OK
         torch.cuda.synchronize()
         assert np.array_equal(y.host().view(np.uint32), expect.view(np.uint32)), kind
 
