@@ -187,7 +187,10 @@ bq_status launch_dequant(const bq::DParams& p, int dev, int sms, cudaStream_t st
   if (s != BQ_OK) return s;
   const int64_t work = p.vec ? (p.nchunks + 3) / 4 + 1 : p.n;
   int64_t want = (work + bq::kDThreads - 1) / bq::kDThreads;
-  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  // up to four waves of resident CTAs: the stores of more CTAs spread over
+  // more of the output at once (8-bit codes: 297 -> 284 us at n = 2^29
+  // bf16; 4-bit codes unchanged)
+  const int64_t cap = static_cast<int64_t>(occ) * sms * 4;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kDThreads, 0, stream, p);

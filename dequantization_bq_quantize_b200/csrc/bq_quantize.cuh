@@ -402,10 +402,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
     fence_mbar_init();
   }
   pdl_release();
-  pdl_wait();  // inputs, codebook and outputs may belong to the previous kernel
   __syncthreads();
 
+  // Under programmatic dependent launch this CTA may start while the previous
+  // kernel on the stream still runs.  The codebook is read and the search
+  // tables are built before waiting for it (the ABI requires the codebook not
+  // to be an output of the immediately preceding library call on the
+  // stream); the input is read and the outputs are written only after the
+  // wait.
   if (warp == 0) {
+    pdl_wait();
     if (lane == 0 && p.full_tiles > 0) {
       int64_t iter = 0;
       for (int64_t tile = blockIdx.x; tile < p.full_tiles; tile += gridDim.x, ++iter) {
@@ -429,6 +435,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
   const int ct = threadIdx.x - 32;
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
+  pdl_wait();
   const int mode = s.tab.mode;
   if (mode == kModeLutF) consumer_main<DT, E, TPB, kModeLutF>(s, p, ct);
   else if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);

@@ -84,6 +84,12 @@ typedef enum bq_dtype {
  *                high nibble of byte i, element 2i+1 in the low nibble (0 if it
  *                does not exist); 256 entries: n bytes, one code per element.
  * Inputs must be finite (non-finite values are outside the contract).
+ * Ordering: the kernel starts under programmatic dependent launch and reads
+ * `code` (to build its search tables) before waiting for the kernel launched
+ * just before it on `stream`; everything else is read and written after that
+ * wait.  So `code` must not be an output of the immediately preceding
+ * library call on the same stream (copies, and kernels of other libraries,
+ * are always complete before it is read).
  */
 BQ_API bq_status bq_quantize_blockwise(const void *x, bq_dtype x_dtype, int64_t n,
                                 int32_t blocksize, const float *code,
