@@ -113,6 +113,28 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return d;
 }
 
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// Packed two-lane signed max / min, NaN-propagating.
+template <int DT>
+__device__ __forceinline__ uint32_t smax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  if constexpr (DT == kBF16) asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  else asm("max.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <int DT>
+__device__ __forceinline__ uint32_t smin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  if constexpr (DT == kBF16) asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  else asm("min.NaN.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Packed two-lane |a| vs |b| max (NaN-propagating) and min; the sign of the
 // result is meaningless and dropped later.
 template <int DT>

@@ -149,11 +149,104 @@ __device__ __forceinline__ uint32_t q4_exact(float x, float id) {
   return t >= 15.0f ? 15u : (t >= 0.0f ? static_cast<uint32_t>(__float2int_rz(t)) : 0u);
 }
 
+// Q4_0 from the block's largest magnitude and its first element m: the fast
+// path when both are usable, else the exact scalar path with the clamps.
+template <int IT>
+__device__ __forceinline__ void encode_q4_from_m(const RawBlk<IT>& r, float amax, float m,
+                                                 uint32_t& dh, uint32_t (&q)[8]) {
+  const float kInf = __int_as_float(0x7f800000);
+  const float d = __fmul_rn(m, -0.125f);
+  const float id = d == 0.0f ? 0.0f : 1.0f / d;  // of either sign here
+  if (amax < kInf && fabsf(id) < kInf) {
+    const uint64_t h2 = pack2(8.5f, 8.5f), m2 = pack2(8388608.0f, 8388608.0f);
+    uint32_t z[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      // scalar products (never contracted), then packed adds
+      const uint64_t t = pack2(__fmul_rn(blk_elem(r, 2 * k), id), __fmul_rn(blk_elem(r, 2 * k + 1), id));
+      float z0, z1;
+      unpack2(add_rz2(add_rn2(t, h2), m2), z0, z1);  // 2^23 + trunc(x * id + 8.5)
+      z[2 * k] = min(__float_as_uint(z0), 0x4B00000Fu);
+      z[2 * k + 1] = min(__float_as_uint(z1), 0x4B00000Fu);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = low_bytes4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
+      const uint32_t hi = low_bytes4(z[16 + 4 * i], z[17 + 4 * i], z[18 + 4 * i], z[19 + 4 * i]);
+      q[i] = lo | (hi << 4);  // every byte of lo and hi is at most 15
+    }
+    dh = half_bits(d);
+  } else {
+    // the first strictly larger magnitude, starting below every magnitude;
+    // NaN never wins.  Magnitudes compare as integers (the order of the
+    // absolute bits of non-NaN floats), with NaN excluded explicitly.
+    int32_t best = -1;
+    float ms = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float v = blk_elem(r, j);
+      const int32_t mag = static_cast<int32_t>(__float_as_uint(v) & 0x7FFFFFFFu);
+      if (mag <= 0x7F800000 && mag > best) {
+        best = mag;
+        ms = v;
+      }
+    }
+    const float ds = __fmul_rn(ms, -0.125f);
+    const float ids = ds == 0.0f ? 0.0f : 1.0f / ds;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = low_bytes4(q4_exact(blk_elem(r, 4 * i), ids),
+                                     q4_exact(blk_elem(r, 4 * i + 1), ids),
+                                     q4_exact(blk_elem(r, 4 * i + 2), ids),
+                                     q4_exact(blk_elem(r, 4 * i + 3), ids));
+      const uint32_t hi = low_bytes4(q4_exact(blk_elem(r, 16 + 4 * i), ids),
+                                     q4_exact(blk_elem(r, 17 + 4 * i), ids),
+                                     q4_exact(blk_elem(r, 18 + 4 * i), ids),
+                                     q4_exact(blk_elem(r, 19 + 4 * i), ids));
+      q[i] = lo | (hi << 4);
+    }
+    dh = half_bits(ds);
+  }
+}
+
 // Encode one block: dh = fp16 bits of d; q = the block's quant bytes
 // (8 words for Q8_0, 4 for Q4_0) in memory order.
 template <int KIND, int IT>
 __device__ __forceinline__ void encode_block(const RawBlk<IT>& r, uint32_t& dh, uint32_t (&q)[8]) {
   const float kInf = __int_as_float(0x7f800000);
+  if constexpr (KIND == kQ4_0 && IT != kF32) {
+    // 16-bit inputs: packed signed max and min give the largest magnitude
+    // and, unless +amax and -amax both occur, the sign of every element that
+    // has it - so the first such element is known without a search
+    uint32_t mx[8], mn[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      mx[i] = smax2<IT>(r.w[2 * i], r.w[2 * i + 1]);
+      mn[i] = smin2<IT>(r.w[2 * i], r.w[2 * i + 1]);
+    }
+#pragma unroll
+    for (int st = 4; st >= 1; st >>= 1)
+#pragma unroll
+      for (int i = 0; i < st; ++i) {
+        mx[i] = smax2<IT>(mx[i], mx[i + st]);
+        mn[i] = smin2<IT>(mn[i], mn[i + st]);
+      }
+    const float hi = max_nan(widen_pair_elem<IT>(mx[0], 0), widen_pair_elem<IT>(mx[0], 1));
+    const float lo = min_nan(widen_pair_elem<IT>(mn[0], 0), widen_pair_elem<IT>(mn[0], 1));
+    const float amax = max_nan(hi, -lo);  // NaN if the block holds a NaN
+    float m;
+    if (amax > 0.0f && hi != -lo) {
+      m = hi == amax ? hi : lo;
+    } else {
+      // zero block, a +amax / -amax tie, or NaN: the first element of
+      // largest magnitude by a scan (scanning down, the last match wins)
+      m = 0.0f;
+#pragma unroll
+      for (int j = 31; j >= 0; --j) m = fabsf(blk_elem(r, j)) == amax ? blk_elem(r, j) : m;
+    }
+    encode_q4_from_m(r, amax, m, dh, q);
+    return;
+  }
   const float amax = blk_amax_nan(r);  // NaN if the block holds a NaN
   if constexpr (KIND == kQ8_0) {
     const float d = amax / 127.0f;
@@ -189,64 +282,13 @@ __device__ __forceinline__ void encode_block(const RawBlk<IT>& r, uint32_t& dh, 
                           q8_exact(blk_elem(r, 4 * i + 2), ids), q8_exact(blk_elem(r, 4 * i + 3), ids));
       dh = half_bits(ds);
     }
-  } else {  // kQ4_0
+  } else {  // kQ4_0, fp32 input
     // the first element whose magnitude is amax (scanning down, the last
     // match is the lowest index); meaningful only when amax is finite
     float m = 0.0f;
 #pragma unroll
     for (int j = 31; j >= 0; --j) m = fabsf(blk_elem(r, j)) == amax ? blk_elem(r, j) : m;
-    const float d = __fmul_rn(m, -0.125f);
-    const float id = d == 0.0f ? 0.0f : 1.0f / d;  // of either sign here
-    if (amax < kInf && fabsf(id) < kInf) {
-      const uint64_t h2 = pack2(8.5f, 8.5f), m2 = pack2(8388608.0f, 8388608.0f);
-      uint32_t z[32];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        // scalar products (never contracted), then packed adds
-        const uint64_t t = pack2(__fmul_rn(blk_elem(r, 2 * k), id), __fmul_rn(blk_elem(r, 2 * k + 1), id));
-        float z0, z1;
-        unpack2(add_rz2(add_rn2(t, h2), m2), z0, z1);  // 2^23 + trunc(x * id + 8.5)
-        z[2 * k] = min(__float_as_uint(z0), 0x4B00000Fu);
-        z[2 * k + 1] = min(__float_as_uint(z1), 0x4B00000Fu);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = low_bytes4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
-        const uint32_t hi = low_bytes4(z[16 + 4 * i], z[17 + 4 * i], z[18 + 4 * i], z[19 + 4 * i]);
-        q[i] = lo | (hi << 4);  // every byte of lo and hi is at most 15
-      }
-      dh = half_bits(d);
-    } else {
-      // the first strictly larger magnitude, starting below every magnitude;
-      // NaN never wins.  Magnitudes compare as integers (the order of the
-      // absolute bits of non-NaN floats), with NaN excluded explicitly.
-      int32_t best = -1;
-      float ms = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float v = blk_elem(r, j);
-        const int32_t mag = static_cast<int32_t>(__float_as_uint(v) & 0x7FFFFFFFu);
-        if (mag <= 0x7F800000 && mag > best) {
-          best = mag;
-          ms = v;
-        }
-      }
-      const float ds = __fmul_rn(ms, -0.125f);
-      const float ids = ds == 0.0f ? 0.0f : 1.0f / ds;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = low_bytes4(q4_exact(blk_elem(r, 4 * i), ids),
-                                       q4_exact(blk_elem(r, 4 * i + 1), ids),
-                                       q4_exact(blk_elem(r, 4 * i + 2), ids),
-                                       q4_exact(blk_elem(r, 4 * i + 3), ids));
-        const uint32_t hi = low_bytes4(q4_exact(blk_elem(r, 16 + 4 * i), ids),
-                                       q4_exact(blk_elem(r, 17 + 4 * i), ids),
-                                       q4_exact(blk_elem(r, 18 + 4 * i), ids),
-                                       q4_exact(blk_elem(r, 19 + 4 * i), ids));
-        q[i] = lo | (hi << 4);
-      }
-      dh = half_bits(ds);
-    }
+    encode_q4_from_m(r, amax, m, dh, q);
   }
 }
 

@@ -282,8 +282,9 @@ def test_gguf_torch_helpers():
 
 def _encode_input(nblk, dtype, seed, special=False):
     """N(0, 0.02) blocks, with every 7th block rounded to a grid of 1/64
-    (ties on |x| and exact halves after scaling) and every 11th all zeros
-    (every 22nd starting with -0).  `special` adds blocks with inf, -inf,
+    (ties on |x| and exact halves after scaling), every 11th all zeros
+    (every 22nd starting with -0) and every 17th (from the 4th) drawn from
+    {+-0.5, 0.25, -0.125, 0} (ties between +amax and -amax).  `special` adds blocks with inf, -inf,
     NaN, fp32/bf16 subnormals and magnitudes whose scale reciprocal
     overflows."""
     g = torch.Generator().manual_seed(seed)
@@ -291,6 +292,10 @@ def _encode_input(nblk, dtype, seed, special=False):
     x[::7] = torch.round(x[::7] * 64) / 64
     x[::11] = 0.0
     x[::22, 0] = -0.0
+    # every 17th block: values from {+-0.5, 0.25, -0.125, 0}, so the largest
+    # magnitude occurs with both signs, in random order
+    pick = torch.randint(0, 5, (x[3::17].shape[0], 32), generator=g)
+    x[3::17] = torch.tensor([0.5, -0.5, 0.25, -0.125, 0.0])[pick]
     if special:
         x[1::13, 3] = float("inf")
         x[2::13, 5] = -float("inf")
