@@ -51,6 +51,10 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
+    ap.add_argument("--gguf-kinds", default="",
+                    help="gguf workload: comma-separated types to run (e.g. q4_k,q8_0_encode)")
+    ap.add_argument("--gguf-sizes", default="small,matrix",
+                    help="gguf workload: 'small' (4096 blocks), 'matrix' (4096 x 14336) or both")
     ap.add_argument("--workload", choices=["step", "sweep", "llama", "gguf", "nested", "h2d"], default="step",
                     help="step: the benchmark line; the others: informational tables")
     return ap.parse_args()
@@ -521,26 +525,65 @@ def run_e2e(args, w, names, stream, sh, byts, world, chunks=8):
 
 # ------------------------------------------------------ informational ---
 
+def _capture(body):
+    """A CUDA graph of body() captured on a side stream (body() is run once
+    first, outside the capture)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        body()
+        with torch.cuda.graph(g, stream=side):
+            body()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    return g
+
+
+def _replay_ms(g, times=5):
+    """Median device time (ms) of one replay of graph g."""
+    ts = []
+    for _ in range(times):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sorted(ts)[len(ts) // 2]
+
+
 def _timed(fn, reps, flush=None):
-    """Device time (ms) of one fn() call.  With `flush`, every call is
-    preceded by a write of the flush buffer (larger than L2): `reps` pairs
-    (flush, fn) are queued back to back and the time of `reps` flushes alone
-    is subtracted, so neither host launch latency nor the flush is counted."""
-    def batch(with_fn):
+    """Device time (ms) of one fn() call.  Without `flush`: `reps` calls back
+    to back between two events, divided by reps.  With `flush` (a buffer
+    larger than L2): `reps` pairs (write the flush buffer, fn()) are captured
+    in one CUDA graph and `reps` flushes alone in another; the difference of
+    their replay times, divided by reps, is fn's time with a cold L2 and
+    without host launch gaps."""
+    fn()  # warm
+    torch.cuda.synchronize()
+    if flush is None:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            if flush is not None:
-                flush.zero_()
-            if with_fn:
-                fn()
+            fn()
         e1.record()
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1)
-    batch(True)  # warm
-    if flush is None:
-        return batch(True) / reps
-    return max(0.0, (batch(True) - batch(False)) / reps)
+        return e0.elapsed_time(e1) / reps
+
+    def both():
+        for _ in range(reps):
+            flush.zero_()
+            fn()
+
+    def alone():
+        for _ in range(reps):
+            flush.zero_()
+
+    g1, g0 = _capture(both), _capture(alone)
+    ms = (_replay_ms(g1) - _replay_ms(g0)) / reps
+    del g1, g0
+    return max(ms, 0.0)
 
 
 def _graph_timed(fn, reps=50):
@@ -566,11 +609,11 @@ def _graph_timed(fn, reps=50):
 def run_sweep(args):
     """45 cells: {fp16, bf16, fp32} x {NF4, FP4, dyn8} x bs {32, 64, 256, 1024,
     4096} at n = 8388608 + 37 with one all-zero block; quantize and dequantize
-    (to the input dtype) timed separately with a 512 MiB L2 flush before each
+    (to the input dtype) timed separately with a 320 MiB L2 flush before each
     repetition (the tensors fit in L2)."""
     import dequantization_bq_quantize_b200 as bq
     dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(1 << 29, dtype=torch.uint8, device=dev)
+    flush = torch.empty(320 << 20, dtype=torch.uint8, device=dev)
     cells = []
     ci = 0
     for dtype in ("f16", "bf16", "f32"):
@@ -649,15 +692,21 @@ def run_llama(args):
 def run_gguf(args):
     """Every GGUF block type on two workloads, bf16 target: the Verification
     table's 4096 blocks (fits in L2 and is launch-bound: 50 calls captured in
-    one CUDA graph, replayed) and a 4096 x 14336 weight matrix (a 512 MiB
+    one CUDA graph, replayed) and a 4096 x 14336 weight matrix (a 320 MiB
     flush precedes each call and its time is subtracted)."""
     import dequantization_bq_quantize_b200 as bq
     dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(1 << 29, dtype=torch.uint8, device=dev)
+    flush = torch.empty(320 << 20, dtype=torch.uint8, device=dev)
     peak = measured_peaks()[0]
     rows = []
+    kinds = set(k for k in args.gguf_kinds.split(",") if k)
+    sizes = set(args.gguf_sizes.split(","))
+    want = lambda k: not kinds or k in kinds
+    pick = lambda pairs: [p for p, tag in zip(pairs, ("small", "matrix")) if tag in sizes]
     for kind, (per, bb) in bq.GGUF_TYPES.items():
-        for label, nblk in (("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // per)):
+        if not want(kind):
+            continue
+        for label, nblk in pick((("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // per))):
             blocks = torch.from_numpy(synth.gguf_blocks(nblk, kind, seed=9).reshape(-1)).to(dev)
             y = torch.empty(nblk * per, dtype=torch.bfloat16, device=dev)
             bq.dequant_gguf(kind, blocks, out=y)
@@ -672,8 +721,10 @@ def run_gguf(args):
             del blocks, y
     # the encoders, bf16 input of the same two sizes
     for kind in bq.GGUF_ENCODERS:
+        if not want(kind + "_encode"):
+            continue
         bb = bq.GGUF_TYPES[kind][1]
-        for label, nblk in (("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // 32)):
+        for label, nblk in pick((("4096 blocks", 4096), ("4096x14336", 4096 * 14336 // 32))):
             g = torch.Generator(device=dev)
             g.manual_seed(17)
             x = torch.randn(nblk * 32, generator=g, device=dev).mul_(0.02).to(torch.bfloat16)
