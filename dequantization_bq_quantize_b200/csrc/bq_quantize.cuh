@@ -24,7 +24,9 @@
 //    per instruction with the sm_100 fp32x2 FMA / MUL (no per-element range
 //    check: see div_fast);
 //  - the code from a bucket table (bq_search.cuh): one packed bucket
-//    computation per pair, two shared loads and one compare per element;
+//    computation per pair, one 64-bit shared load and one compare per
+//    element (16-entry tables: each lane reads its own interleaved copy, so
+//    the loads never conflict on banks);
 //  - codes inserted into the output words with bit-field inserts.
 // Blocks whose absmax is outside [2^-60, 2^60] (or not finite), and codebooks
 // without a bucket table, take the safe path: IEEE division where Markstein's
@@ -84,13 +86,6 @@ __device__ __forceinline__ uint32_t bfi(uint32_t field, uint32_t base, int pos, 
 // it is only ever fed addresses computed from tile data loaded after the
 // mbarrier wait (itself after the table build and its barrier): the data
 // dependence keeps it after both.
-template <uint32_t OFF = 0>
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
-  return v;
-}
-
 __device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
   uint2 v;
   asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -122,14 +117,15 @@ struct QOut {
 
 // ------------------------------------------------------ fast encoding -----
 
-// Shared address of lut.e[bucket].  For 16-entry tables `b` is already
-// fma(xn, 15, 1.5 * 2^23) and t_base = &lut.e[0] - 8 * (0x4B400000 - 15), so
-// bits(b) * 8 + t_base addresses the bucket (32-bit wrap-around arithmetic).
-// For 256-entry tables b is xn and t_base = &lut.e[1537].
+// Shared address of the bucket's entry.  For 16-entry tables `b` is already
+// fma(xn, 15, 1.5 * 2^23) and t_base = &lut.r[0][lane % 16] -
+// 128 * (0x4B400000 - 15), so bits(b) * 128 + t_base addresses this lane's
+// copy of the bucket (32-bit wrap-around arithmetic).  For 256-entry tables b
+// is xn and t_base = &lut.e[1537].
 template <int E>
 __device__ __forceinline__ uint32_t lut_addr(float b, uint32_t t_base) {
   if constexpr (E == 16) {
-    return __float_as_uint(b) * 8u + t_base;
+    return __float_as_uint(b) * 128u + t_base;
   } else {
     const uint32_t u = __float_as_uint(b);
     const uint32_t a = u & 0x7fffffffu;
@@ -140,16 +136,9 @@ __device__ __forceinline__ uint32_t lut_addr(float b, uint32_t t_base) {
 }
 
 template <int E>
-__device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut) {
-  if constexpr (E == 16) return smem_u32(lut.e) - 8u * (0x4B400000u - 15u);
+__device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut, int lane) {
+  if constexpr (E == 16) return smem_u32(&lut.r[0][lane & 15]) - 128u * (0x4B400000u - 15u);
   else return smem_u32(lut.e) + 8u * 1537u;
-}
-
-// Base of the split arrays of 16-entry tables (0 otherwise, unused).
-template <int E>
-__device__ __forceinline__ uint32_t lut_base_split(const Lut<E>& lut) {
-  if constexpr (E == 16) return smem_u32(lut.a) - 4u * (0x4B400000u - 15u);
-  else return 0u;
 }
 
 // Weight of element j within its 16-bit half of the output: a half holds 4
@@ -167,7 +156,8 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 
 // Fast path: the block's reciprocal is valid for Markstein's form and the
 // codebook has a bucket table.  Two elements per packed division and bucket
-// computation; one 64-bit table load per element.
+// computation; one 64-bit table load per element (conflict-free for 16-entry
+// tables: each lane reads its own copy).
 //  kModeLut:  code = q >= t ? code1 : code0, inserted with a bit-field insert.
 //  kModeLutF: H = sat(fma(q, 2^60, K)) is exactly [q >= t]; code = C + H is
 //             accumulated in fp32 into 16-bit halves (2^23 + sum of
@@ -176,8 +166,7 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 //             bytes are merged with one byte permute per word.
 template <int DT, int E, int MODE>
 __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
-                                            uint32_t t_base, uint32_t a_base,
-                                            uint32_t (&ow)[QOut<DT, E>::NW]) {
+                                            uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
   using O = QOut<DT, E>;
   constexpr int NH = 2 * O::NW;                 // 16-bit halves
   constexpr int PER_HALF = O::EPT / NH;         // elements per half (4 or 2)
@@ -192,15 +181,7 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
     if constexpr (E == 16)
       unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
     const uint2 e0 = lds_u64(lut_addr<E>(b0, t_base));
-    uint2 e1;
-    if constexpr (E == 16) {
-      // second element from the split 32-bit arrays (lut.b is 128 bytes past
-      // lut.a): a_base = &lut.a[0] - 4 * (0x4B400000 - 15)
-      const uint32_t ad1 = __float_as_uint(b1) * 4u + a_base;
-      e1 = make_uint2(lds_u32<0>(ad1), lds_u32<128>(ad1));
-    } else {
-      e1 = lds_u64(lut_addr<E>(b1, t_base));
-    }
+    const uint2 e1 = lds_u64(lut_addr<E>(b1, t_base));
     const int j0 = 2 * i, j1 = 2 * i + 1;
     if constexpr (MODE == kModeLutF) {
       const float h0 = fma_sat(q0, kSelScale, __uint_as_float(e0.x));
@@ -251,7 +232,7 @@ __device__ __forceinline__ void encode_safe(const uint32_t (&w)[kThreadWords], c
 template <int DT, int E, int TPB, int MODE>
 __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uint32_t tile,
                                               int st, uint32_t par, uint32_t iter, int ct,
-                                              uint32_t t_base, uint32_t a_base) {
+                                              uint32_t t_base) {
   using O = QOut<DT, E>;
   constexpr int TE = kTileBytes / ElemBytes<DT>::value;
   constexpr int BPT = kQConsumers / TPB;
@@ -321,7 +302,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   // per-element condition is not needed, see div_fast); NaN fails both tests
   constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
-  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, a_base, ow);
+  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, ow);
   else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
@@ -367,14 +348,13 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 template <int DT, int E, int TPB, int MODE>
 __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int ct) {
   constexpr int BPT = kQConsumers / TPB;
-  const uint32_t t_base = lut_base<E>(s.lut);
-  const uint32_t a_base = lut_base_split<E>(s.lut);
+  const uint32_t t_base = lut_base<E>(s.lut, ct & 31);
   const uint32_t ntiles = static_cast<uint32_t>(p.full_tiles);  // < 2^24 (host check)
   uint32_t iter = 0;
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
     const int st = static_cast<int>(iter % kStages);
     const uint32_t par = (iter / kStages) & 1u;
-    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base, a_base)) break;
+    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base)) break;
   }
   // what the tiles did not cover: one quantization block per warp
   const int lane = ct & 31, cw = ct >> 5;
