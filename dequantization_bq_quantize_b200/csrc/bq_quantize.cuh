@@ -164,7 +164,11 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 //             code * weight, every value an exact integer below 2^24; the
 //             first element of a half brings the 2^23), and the halves' low
 //             bytes are merged with one byte permute per word.
-template <int DT, int E, int MODE>
+//  REMAP (16-entry tables like FP4, whose +-0 pair makes one step of two):
+//             the table holds ranks of the distinct values, which step by
+//             one; each nibble >= 8 then gets 1 added (ranks 8..14 -> codes
+//             9..15), three instructions per 8 codes.
+template <int DT, int E, int MODE, bool REMAP>
 __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
                                             uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
   using O = QOut<DT, E>;
@@ -204,6 +208,13 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
 #pragma unroll
     for (int k = 0; k < O::NW; ++k)
       ow[k] = __byte_perm(__float_as_uint(hacc[2 * k]), __float_as_uint(hacc[2 * k + 1]), 0x5410);
+    if constexpr (E == 16) {
+      // ranks 8..14 -> codes 9..15: add bit 3 of every nibble to that nibble
+      if constexpr (REMAP) {
+#pragma unroll
+        for (int k = 0; k < O::NW; ++k) ow[k] += (ow[k] >> 3) & 0x11111111u;
+      }
+    }
   }
 }
 
@@ -229,7 +240,7 @@ __device__ __forceinline__ void encode_safe(const uint32_t (&w)[kThreadWords], c
 
 // --------------------------------------------------- one tile (consumer) --
 
-template <int DT, int E, int TPB, int MODE>
+template <int DT, int E, int TPB, int MODE, bool REMAP>
 __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uint32_t tile,
                                               int st, uint32_t par, uint32_t iter, int ct,
                                               uint32_t t_base) {
@@ -302,7 +313,8 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   // per-element condition is not needed, see div_fast); NaN fails both tests
   constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
-  if (fast) encode_fast<DT, E, kBucket ? MODE : kModeLut>(w, make_scale_fast(A), t_base, ow);
+  if (fast)
+    encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP>(w, make_scale_fast(A), t_base, ow);
   else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
@@ -345,7 +357,7 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 
 // ------------------------------------------------------------- kernel -----
 
-template <int DT, int E, int TPB, int MODE>
+template <int DT, int E, int TPB, int MODE, bool REMAP = false>
 __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int ct) {
   constexpr int BPT = kQConsumers / TPB;
   const uint32_t t_base = lut_base<E>(s.lut, ct & 31);
@@ -354,7 +366,7 @@ __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
     const int st = static_cast<int>(iter % kStages);
     const uint32_t par = (iter / kStages) & 1u;
-    if (!quantize_tile<DT, E, TPB, MODE>(s, p, tile, st, par, iter, ct, t_base)) break;
+    if (!quantize_tile<DT, E, TPB, MODE, REMAP>(s, p, tile, st, par, iter, ct, t_base)) break;
   }
   // what the tiles did not cover: one quantization block per warp
   const int lane = ct & 31, cw = ct >> 5;
@@ -417,7 +429,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   pdl_wait();
   const int mode = s.tab.mode;
-  if (mode == kModeLutF) consumer_main<DT, E, TPB, kModeLutF>(s, p, ct);
+  // REMAP: FP4-like 16-entry tables, float select over ranks (bq_search.cuh)
+  if (mode == kModeLutF && E == 16 && s.tab.remap8)
+    consumer_main<DT, E, TPB, kModeLutF, E == 16>(s, p, ct);
+  else if (mode == kModeLutF) consumer_main<DT, E, TPB, kModeLutF>(s, p, ct);
   else if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);
   else if (mode == kModeBsearch) consumer_main<DT, E, TPB, kModeBsearch>(s, p, ct);
   else consumer_main<DT, E, TPB, kModeScan>(s, p, ct);

@@ -476,11 +476,19 @@ def test_division_fp32_random(probes):
 
 
 # search forms: 0 = bucket table, integer select; 3 = bucket table, float
-# select (codes step by one at every threshold); FP4's +-0 pair makes one step 2
-@pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 0), ("dyn8", 3)])
+# select (codes step by one at every threshold; FP4's +-0 pair, the one step
+# of two, is handled by selecting over ranks and adding 1 from rank 8 on).
+# "dup34" repeats entries 3 and 4, a step of two that only the integer
+# select handles.
+_DUP34 = TABLES["nf4"].copy()
+_DUP34[4] = _DUP34[3]
+
+
+@pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 3), ("dyn8", 3),
+                                              ("dup34", 0)])
 @pytest.mark.parametrize("force", [-1, 1], ids=["chosen", "bisection"])
 def test_search_exhaustive(probes, name, expect_mode, force):
-    table = TABLES[name]
+    table = _DUP34 if name == "dup34" else TABLES[name]
     code = code_dev(table)
     mode = ctypes.c_int(-1)
     mm, fa, fb = _outs()
