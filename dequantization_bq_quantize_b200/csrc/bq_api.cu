@@ -238,7 +238,8 @@ bq_status launch_gguf(const bq::GParams& p, int dev, int sms, cudaStream_t strea
   constexpr int kStep = bq::GStep<KIND>::value;
   const int64_t steps = (p.n_blocks + kStep - 1) / kStep;
   int64_t want = (steps + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
-  const int64_t cap = static_cast<int64_t>(occ) * sms;
+  // up to four waves of resident CTAs (Q4_K 4096 x 14336: 31.8 -> 28.7 us)
+  const int64_t cap = static_cast<int64_t>(occ) * sms * 4;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   cudaError_t e = launch_pdl(kernel, static_cast<int>(want), bq::kGThreads, 0, stream, p);
@@ -294,6 +295,7 @@ bq_status launch_gguf_encode(const bq::GEParams& p, int dev, int sms, cudaStream
   if (s != BQ_OK) return s;
   const int64_t steps = (p.n_blocks + 31) / 32;
   int64_t want = (steps + bq::kGThreads / 32 - 1) / (bq::kGThreads / 32);
+  // one wave of resident CTAs (four waves measured slower for the encoders)
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
