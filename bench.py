@@ -371,7 +371,8 @@ def run_ours(args, rank, world, local):
         gbs = byts[k] / (ms / 1e3) / 1e9
         kern[k] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
                    "bytes": byts[k]}
-    dom = "quantize" if "quantize" in kern else names[0]
+    # the dominant kernel: the one that takes the longest in the step
+    dom = max(kern, key=lambda k: kern[k]["ms"])
     kname = {"quantize": "quantize_kernel<bf16,nf4,bs64>", "dequantize":
              "dequant_kernel<nf4,bf16>", "q8_0": "gguf_kernel<q8_0,bf16>",
              "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
