@@ -50,7 +50,7 @@ extern "C" {
 typedef enum bq_status {
     BQ_OK = 0,
     BQ_ERR_INVALID_ARG = 1,   /* bad size, pointer, blocksize or codebook length */
-    BQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement     */
+    BQ_ERR_UNSUPPORTED = 2,   /* valid request this library does not implement   */
     BQ_ERR_CUDA = 3           /* a CUDA call failed; see bq_last_cuda_error()    */
 } bq_status;
 
