@@ -94,33 +94,37 @@ __device__ __forceinline__ uint2 load_codes(const uint8_t* __restrict__ q, int64
 // table reads are asm with no memory dependence: their addresses come from
 // code bytes loaded from global memory after the table was built and
 // __syncthreads, and that data dependence keeps them after the build.
-template <int E>
+// STRIDE: bytes between consecutive table entries (8 / 4 for a plain table;
+// 128 for a table replicated per lane, t_base then pointing at this lane's
+// copy).
+template <int E, int STRIDE = (E == 16 ? 8 : 4)>
 __device__ __forceinline__ void decode_pair(uint2 c, int k, uint32_t t_base, uint64_t a2,
                                             float& v0, float& v1) {
   if constexpr (E == 16) {
     // byte k of the chunk's code word: elements 2k (high nibble), 2k+1 (low)
     const uint32_t byte = __byte_perm(c.x, 0u, 0x4440u + k);
     uint2 pr;
-    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(pr.x), "=r"(pr.y) : "r"(t_base + byte * 8u));
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(pr.x), "=r"(pr.y) : "r"(t_base + byte * STRIDE));
     unpack2(mul2(pack2(__uint_as_float(pr.x), __uint_as_float(pr.y)), a2), v0, v1);
   } else {
     const uint32_t word = k < 2 ? c.x : c.y;
     const uint32_t b0 = __byte_perm(word, 0u, 0x4440u + 2 * (k & 1));
     const uint32_t b1 = __byte_perm(word, 0u, 0x4441u + 2 * (k & 1));
     float c0, c1;
-    asm("ld.shared.f32 %0, [%1];" : "=f"(c0) : "r"(t_base + b0 * 4u));
-    asm("ld.shared.f32 %0, [%1];" : "=f"(c1) : "r"(t_base + b1 * 4u));
+    asm("ld.shared.f32 %0, [%1];" : "=f"(c0) : "r"(t_base + b0 * STRIDE));
+    asm("ld.shared.f32 %0, [%1];" : "=f"(c1) : "r"(t_base + b1 * STRIDE));
     unpack2(mul2(pack2(c0, c1), a2), v0, v1);
   }
 }
 
-template <int E, int OT>
+template <int E, int OT, int STRIDE = (E == 16 ? 8 : 4)>
 __device__ __forceinline__ uint4 decode_chunk(uint2 c, float A, uint32_t t_base) {
   constexpr int CE = DTraits<E, OT>::CE;
   const uint64_t a2 = pack2(A, A);
   float v[CE];
 #pragma unroll
-  for (int k = 0; k < CE / 2; ++k) decode_pair<E>(c, k, t_base, a2, v[2 * k], v[2 * k + 1]);
+  for (int k = 0; k < CE / 2; ++k)
+    decode_pair<E, STRIDE>(c, k, t_base, a2, v[2 * k], v[2 * k + 1]);
   if constexpr (OT == kF32) {
     return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
                       __float_as_uint(v[3]));

@@ -1,0 +1,184 @@
+// bq_dequant_stream.cuh - blockwise dequantization with the code stream
+// staged through shared memory (sm_100a).
+//
+// Same result as dequant_kernel (bq_dequant.cuh): y_i = narrow(RN(code[idx_i]
+// * absmax[i / blocksize])), the inverse map of "bitsandbytes PR #2052".
+//
+// Why a second kernel.  Dequantization writes about four times the bytes it
+// reads.  In dequant_kernel every warp loads its codes and scales, waits for
+// them, decodes and stores, so each iteration's stores wait behind the
+// global-load latency of its own loads: at n = 2^29 bf16 it takes 254 us,
+// and without any loads the same stores take 158 us.  Here the loads run
+// ahead: a persistent grid of 288-thread CTAs, one producer lane streaming
+// each tile's codes (4 KiB for 4-bit, 8 KiB for 8-bit codes of 8192
+// elements) and its slice of absmax into a 4-stage shared-memory ring with
+// 1-D bulk copies (cp.async.bulk, no multicast) completed by mbarrier
+// transaction counts, and 8 consumer warps decoding from shared memory.  A
+// consumer warp owns 128 consecutive 16-byte output chunks of the tile, so
+// its four stores per lane are 2 KiB of contiguous output, and decodes with
+// a per-lane copy of the table (below), free of bank conflicts.
+//
+// Used for 4-bit codes with plain statistics when codes, absmax and y are
+// 16-byte aligned and blocksize <= 2048 (so a tile's absmax slice is a whole
+// number of 16-byte units); the elements after the last whole tile are done
+// one per thread from global memory.  (The template also covers 8-bit codes,
+// which measured faster on dequant_kernel.)  Every mbarrier wait gives up after a bounded time,
+// sets a bit of the device fault word (4: consumer, 8: producer) and leaves
+// the kernel instead of hanging.
+#pragma once
+
+#include "bq_dequant.cuh"
+
+namespace bq {
+
+constexpr int kSTile = 8192;                          // elements per tile
+constexpr int kSStages = 4;
+constexpr int kSConsumerWarps = 8;
+constexpr int kSThreads = 32 * (kSConsumerWarps + 1);
+
+// The decode table is replicated per lane so that its lookups never conflict
+// on banks (the codes of normal data are close to equiprobable, so a warp's
+// lookups hit random entries): 4-bit codes read 8-byte pairs, copy s = lane %
+// 16 of pair b at tr + 128 b + 8 s (one 128-byte row per pair, copy s in bank
+// pair s); 8-bit codes read 4-byte values, copy l = lane of value b at
+// tr + 128 b + 4 l.  32 KiB either way.  At n = 2^29 bf16 NF4 inside the
+// benchmark step: 251 us (dequant_kernel) -> 236 us.
+template <int E>
+struct SSmem {
+  static constexpr int CODE_BYTES = E == 16 ? kSTile / 2 : kSTile;
+  uint8_t codes[kSStages][CODE_BYTES];                 // 16-byte aligned
+  float amax[kSStages][kSTile / 32];                   // blocksize >= 32
+  uint64_t full[kSStages];
+  uint64_t empty[kSStages];
+  float code[E];
+  float tr[256 * 32];
+};
+
+template <int E>
+constexpr size_t ssmem_bytes() { return sizeof(SSmem<E>) + 128; }
+
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
+// addresses 16-byte aligned and bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int QB>
+__device__ __forceinline__ uint2 smem_codes(const uint8_t* base, int chunk) {
+  if constexpr (QB == 8) return *reinterpret_cast<const uint2*>(base + 8 * chunk);
+  else if constexpr (QB == 4) return make_uint2(*reinterpret_cast<const uint32_t*>(base + 4 * chunk), 0u);
+  else return make_uint2(*reinterpret_cast<const unsigned short*>(base + 2 * chunk), 0u);
+}
+
+template <int E, int OT>
+__global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams p, int64_t ntiles) {
+  using T = DTraits<E, OT>;
+  constexpr int CHUNKS = kSTile / T::CE;                 // 16-byte output chunks per tile
+  constexpr int PER_WARP = CHUNKS / kSConsumerWarps;     // 128 or 256
+  constexpr int PER_LANE = PER_WARP / 32;                // 4 or 8
+  constexpr int CODE_BYTES = SSmem<E>::CODE_BYTES;
+  extern __shared__ uint8_t dsmem_raw[];
+  SSmem<E>& s = *reinterpret_cast<SSmem<E>*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 127) & ~static_cast<uintptr_t>(127));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int abs_per_tile = kSTile >> p.bs_log2;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], kSConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  pdl_release();
+  __syncthreads();
+
+  if (warp == kSConsumerWarps) {  // producer
+    pdl_wait();  // codes and absmax may be written by the previous kernel
+    if (lane == 0) {
+      int64_t iter = 0;
+      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
+        const int st = static_cast<int>(iter % kSStages);
+        if (iter >= kSStages) {
+          const uint32_t par = static_cast<uint32_t>(((iter / kSStages) & 1) ^ 1);
+          if (!mbar_wait_bounded(&s.empty[st], par)) {
+            record_fault(8u);
+            break;
+          }
+        }
+        const uint32_t abytes = 4u * static_cast<uint32_t>(abs_per_tile);
+        mbar_arrive_expect_tx(&s.full[st], CODE_BYTES + abytes);
+        bulk_load(s.codes[st], p.q + tile * CODE_BYTES, CODE_BYTES, &s.full[st]);
+        bulk_load(s.amax[st], p.absmax + tile * abs_per_tile, abytes, &s.full[st]);
+      }
+      // every copy issued must have landed before the CTA may exit
+      for (int64_t j = iter > kSStages ? iter - kSStages : 0; j < iter; ++j)
+        (void)mbar_wait_bounded(&s.full[j % kSStages], static_cast<uint32_t>((j / kSStages) & 1));
+    }
+    return;
+  }
+
+  // consumers: the codebook (pair table for 4-bit codes), then the tiles
+  const int ct = threadIdx.x;  // 0..255
+  pdl_wait();
+  for (int i = ct; i < E; i += 32 * kSConsumerWarps) s.code[i] = p.code[i];
+  named_sync(1, 32 * kSConsumerWarps);
+  if constexpr (E == 16) {
+    // entry (b, copy c) = (code[b >> 4], code[b & 15]) at float index 32 b + 2 c
+    for (int i = ct; i < 256 * 16; i += 32 * kSConsumerWarps) {
+      const int b = i >> 4, c = i & 15;
+      s.tr[32 * b + 2 * c] = s.code[b >> 4];
+      s.tr[32 * b + 2 * c + 1] = s.code[b & 15];
+    }
+  } else {
+    for (int i = ct; i < 256 * 32; i += 32 * kSConsumerWarps) s.tr[i] = s.code[i >> 5];
+  }
+  named_sync(1, 32 * kSConsumerWarps);
+  const uint32_t t_base = smem_u32(s.tr) + (E == 16 ? 8u * (lane & 15) : 4u * lane);
+
+  uint4* y4 = static_cast<uint4*>(p.y);
+  int64_t iter = 0;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
+    const int st = static_cast<int>(iter % kSStages);
+    // warp-uniform: if any lane gives up, the whole warp leaves together
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((iter / kSStages) & 1)))) {
+      if (lane == 0) record_fault(4u);
+      break;  // the producer gives up too, on the stage this warp never frees
+    }
+    uint2 c[PER_LANE];
+    float A[PER_LANE];
+#pragma unroll
+    for (int u = 0; u < PER_LANE; ++u) {
+      const int ch = warp * PER_WARP + u * 32 + lane;
+      c[u] = smem_codes<T::QB>(s.codes[st], ch);
+      A[u] = s.amax[st][(ch * T::CE) >> p.bs_log2];
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp's part is in registers
+    const int64_t first = tile * CHUNKS + warp * PER_WARP + lane;
+#pragma unroll
+    for (int u = 0; u < PER_LANE; ++u)
+      y4[first + u * 32] = decode_chunk<E, OT, 128>(c[u], A[u], t_base);
+  }
+
+  // the elements after the last whole tile, one per thread
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * (32 * kSConsumerWarps) + ct;
+  const int64_t gsz = static_cast<int64_t>(gridDim.x) * (32 * kSConsumerWarps);
+  for (int64_t i = ntiles * kSTile + gtid; i < p.n; i += gsz) {
+    uint32_t idx;
+    if constexpr (E == 16) {
+      const uint32_t byte = p.q[i >> 1];
+      idx = (i & 1) ? (byte & 15u) : (byte >> 4);
+    } else {
+      idx = p.q[i];
+    }
+    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], __ldg(p.absmax + (i >> p.bs_log2))));
+  }
+}
+
+}  // namespace bq

@@ -342,7 +342,8 @@ BQ_API const char *bq_last_cuda_error(void);
  * bounded time instead of hanging, set a bit here and return; results of that
  * launch are then invalid.  Reads the word of the current device (this call
  * SYNCHRONIZES the device), stores it in *fault and, if reset != 0, clears it.
- * 0 means no fault was recorded.
+ * 0 means no fault was recorded.  Bits: 1 / 2 quantize consumer / producer
+ * wait, 4 / 8 dequantize consumer / producer wait.
  */
 BQ_API bq_status bq_device_fault(uint32_t *fault, int32_t reset);
 
