@@ -374,7 +374,7 @@ def run_ours(args, rank, world, local):
     # the dominant kernel: the one that takes the longest in the step
     dom = max(kern, key=lambda k: kern[k]["ms"])
     kname = {"quantize": "quantize_kernel<bf16,nf4,bs64>", "dequantize":
-             "dequant_kernel<nf4,bf16>", "q8_0": "gguf_kernel<q8_0,bf16>",
+             "dequant_stream_kernel<nf4,bf16>", "q8_0": "gguf_kernel<q8_0,bf16>",
              "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
     roof = {"bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak, "unit": "GB/s",
             "frac": kern[dom]["frac"], "traffic": recorded_traffic(kname),
