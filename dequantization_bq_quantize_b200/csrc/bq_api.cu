@@ -204,11 +204,11 @@ bq_status dispatch_dequant(const bq::DParams& p, int entries, int dev, int sms, 
   return launch_dequant<256, OT, NESTED>(p, dev, sms, st);
 }
 
-template <int E, int OT>
+template <int E, int OT, bool NESTED>
 bq_status launch_dequant_stream(const bq::DParams& p, int64_t ntiles, int dev, int sms,
                                 cudaStream_t stream) {
   static KernelSlot slot;
-  auto kernel = bq::dequant_stream_kernel<E, OT>;
+  auto kernel = bq::dequant_stream_kernel<E, OT, NESTED>;
   constexpr size_t smem = bq::ssmem_bytes<E>();
   int occ = 1;
   bq_status s = kernel_occupancy(slot, kernel, dev, bq::kSThreads, smem, &occ);
@@ -236,17 +236,23 @@ bq_status dequant_entry(bq::DParams p, int64_t n, int32_t blocksize, int32_t cod
   const int qb = code_entries == 16 ? ce / 2 : ce;
   p.vec = aligned(p.y, 16) && aligned(p.q, qb);
   p.nchunks = p.vec ? n / ce : 0;
-  // 4-bit codes with plain statistics, 16-byte aligned buffers, at least one
-  // whole tile and a tile's absmax slice a whole number of 16-byte units:
-  // stream the codes through shared memory.  (8-bit codes measured faster on
-  // dequant_kernel: their 8 KiB stages and 32-copy table leave 3 CTAs per SM.)
-  if (!NESTED && code_entries == 16 && aligned(p.y, 16) && aligned(p.q, 16) &&
-      aligned(p.absmax, 16) && blocksize <= 2048 && n >= bq::kSTile) {
+  // 4-bit codes, 16-byte aligned buffers, at least one whole tile, and a
+  // tile's statistics slice a whole number of 16-byte units (plain: 4-byte
+  // scales, blocksize <= 2048; nested: 1-byte codes, blocksize <= 512, and
+  // one second-level scale per tile): stream the codes through shared
+  // memory.  (8-bit codes measured faster on dequant_kernel: their 8 KiB
+  // stages and 32-copy table leave 3 CTAs per SM.)
+  const bool stream_ok =
+      NESTED ? (aligned(p.qa, 16) && blocksize <= 512 &&
+                int64_t{blocksize} << p.bs2_log2 >= bq::kSTile)
+             : (aligned(p.absmax, 16) && blocksize <= 2048);
+  if (stream_ok && code_entries == 16 && aligned(p.y, 16) && aligned(p.q, 16) &&
+      n >= bq::kSTile) {
     const int64_t ntiles = n / bq::kSTile;
     switch (y_dtype) {
-      case BQ_F32: return launch_dequant_stream<16, bq::kF32>(p, ntiles, dev, info.sms, stream);
-      case BQ_F16: return launch_dequant_stream<16, bq::kF16>(p, ntiles, dev, info.sms, stream);
-      default: return launch_dequant_stream<16, bq::kBF16>(p, ntiles, dev, info.sms, stream);
+      case BQ_F32: return launch_dequant_stream<16, bq::kF32, NESTED>(p, ntiles, dev, info.sms, stream);
+      case BQ_F16: return launch_dequant_stream<16, bq::kF16, NESTED>(p, ntiles, dev, info.sms, stream);
+      default: return launch_dequant_stream<16, bq::kBF16, NESTED>(p, ntiles, dev, info.sms, stream);
     }
   }
   switch (y_dtype) {

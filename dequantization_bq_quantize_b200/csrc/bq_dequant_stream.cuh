@@ -47,10 +47,12 @@ template <int E>
 struct SSmem {
   static constexpr int CODE_BYTES = E == 16 ? kSTile / 2 : kSTile;
   uint8_t codes[kSStages][CODE_BYTES];                 // 16-byte aligned
-  float amax[kSStages][kSTile / 32];                   // blocksize >= 32
+  float amax[kSStages][kSTile / 32];                   // blocksize >= 32; NESTED:
+                                                       // the statistics codes as bytes
   uint64_t full[kSStages];
   uint64_t empty[kSStages];
   float code[E];
+  float code2[256];                                    // NESTED only
   float tr[256 * 32];
 };
 
@@ -74,7 +76,13 @@ __device__ __forceinline__ uint2 smem_codes(const uint8_t* base, int chunk) {
   else return make_uint2(*reinterpret_cast<const unsigned short*>(base + 2 * chunk), 0u);
 }
 
-template <int E, int OT>
+// NESTED (compressed statistics): the stage's statistics slot holds the
+// tile's statistics codes (one byte per block; blocksize <= 512 keeps them a
+// whole number of 16-byte units), and the tile's second-level scale
+// (blocksize * blocksize2 >= the tile, so one per tile) comes from global
+// memory, fetched a tile ahead.  A_b = RN(code2[qa_b] * absmax2), as in
+// dequant_kernel.
+template <int E, int OT, bool NESTED>
 __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams p, int64_t ntiles) {
   using T = DTraits<E, OT>;
   constexpr int CHUNKS = kSTile / T::CE;                 // 16-byte output chunks per tile
@@ -110,10 +118,13 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
             break;
           }
         }
-        const uint32_t abytes = 4u * static_cast<uint32_t>(abs_per_tile);
+        const uint32_t abytes = (NESTED ? 1u : 4u) * static_cast<uint32_t>(abs_per_tile);
         mbar_arrive_expect_tx(&s.full[st], CODE_BYTES + abytes);
         bulk_load(s.codes[st], p.q + tile * CODE_BYTES, CODE_BYTES, &s.full[st]);
-        bulk_load(s.amax[st], p.absmax + tile * abs_per_tile, abytes, &s.full[st]);
+        if constexpr (NESTED)
+          bulk_load(s.amax[st], p.qa + tile * abs_per_tile, abytes, &s.full[st]);
+        else
+          bulk_load(s.amax[st], p.absmax + tile * abs_per_tile, abytes, &s.full[st]);
       }
       // every copy issued must have landed before the CTA may exit
       for (int64_t j = iter > kSStages ? iter - kSStages : 0; j < iter; ++j)
@@ -126,6 +137,8 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
   const int ct = threadIdx.x;  // 0..255
   pdl_wait();
   for (int i = ct; i < E; i += 32 * kSConsumerWarps) s.code[i] = p.code[i];
+  if constexpr (NESTED)
+    for (int i = ct; i < 256; i += 32 * kSConsumerWarps) s.code2[i] = p.code2[i];
   named_sync(1, 32 * kSConsumerWarps);
   if constexpr (E == 16) {
     // entry (b, copy c) = (code[b >> 4], code[b & 15]) at float index 32 b + 2 c
@@ -141,8 +154,21 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
   const uint32_t t_base = smem_u32(s.tr) + (E == 16 ? 8u * (lane & 15) : 4u * lane);
 
   uint4* y4 = static_cast<uint4*>(p.y);
+  // NESTED: second-level scale of the tile (block index >> bs2_log2 of the
+  // tile's first block), loaded one tile ahead
+  const int sh2 = p.bs2_log2 + p.bs_log2;
+  float a2_next = 0.0f;
+  if constexpr (NESTED)
+    if (static_cast<int64_t>(blockIdx.x) < ntiles)
+      a2_next = __ldg(p.absmax2 + ((static_cast<int64_t>(blockIdx.x) * kSTile) >> sh2));
   int64_t iter = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
+    float a2 = 0.0f;
+    if constexpr (NESTED) {
+      a2 = a2_next;
+      const int64_t nt = tile + gridDim.x;
+      if (nt < ntiles) a2_next = __ldg(p.absmax2 + ((nt * kSTile) >> sh2));
+    }
     const int st = static_cast<int>(iter % kSStages);
     // warp-uniform: if any lane gives up, the whole warp leaves together
     if (!__all_sync(0xffffffffu,
@@ -156,7 +182,12 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
     for (int u = 0; u < PER_LANE; ++u) {
       const int ch = warp * PER_WARP + u * 32 + lane;
       c[u] = smem_codes<T::QB>(s.codes[st], ch);
-      A[u] = s.amax[st][(ch * T::CE) >> p.bs_log2];
+      if constexpr (NESTED) {
+        const uint32_t qa = reinterpret_cast<const uint8_t*>(s.amax[st])[(ch * T::CE) >> p.bs_log2];
+        A[u] = __fmul_rn(s.code2[qa], a2);
+      } else {
+        A[u] = s.amax[st][(ch * T::CE) >> p.bs_log2];
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp's part is in registers
@@ -177,7 +208,11 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
     } else {
       idx = p.q[i];
     }
-    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], __ldg(p.absmax + (i >> p.bs_log2))));
+    const int64_t b = i >> p.bs_log2;
+    float A;
+    if constexpr (NESTED) A = __fmul_rn(s.code2[p.qa[b]], __ldg(p.absmax2 + (b >> p.bs2_log2)));
+    else A = __ldg(p.absmax + b);
+    store_elem<OT>(p.y, i, __fmul_rn(s.code[idx], A));
   }
 }
 

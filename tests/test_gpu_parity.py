@@ -523,7 +523,7 @@ def _oracle_nested(xh, dtype, bs, bs2, n, ydtype, table=None):
 
 
 @pytest.mark.parametrize("dtype,bs,bs2", [("bf16", 64, 256), ("f16", 4096, 256), ("f32", 32, 256),
-                                          ("bf16", 256, 32), ("f16", 32, 4096)])
+                                          ("bf16", 256, 32), ("f16", 32, 4096), ("bf16", 32, 64)])
 def test_nested_statistics_parity(dtype, bs, bs2):
     """Compressed statistics: the absmax array quantized with the dynamic
     8-bit table in blocks of blocksize2, against the same composition of
