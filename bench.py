@@ -266,10 +266,38 @@ def cpu_baseline(n, nblk, x_cpu):
     oracle.dequant_q4_0(q4, "bf16")
     dt = time.perf_counter() - t0
     byts = sum(step_bytes(n_s, nblk_s).values())
+    # one thread, the plain oracle calls: median of 3 on the first 2^23 elements
+    n_1 = min(n_s, 1 << 23)
+    t1 = []
+    for _ in range(3):
+        t = time.perf_counter()
+        a1, q1 = oracle.quantize_blockwise(xb[:n_1], "bf16", BS, nf4)
+        oracle.dequantize_blockwise(q1, a1, n_1, BS, nf4, "bf16")
+        t1.append(time.perf_counter() - t)
+    one = 2 * quant_bytes(n_1, BS) / statistics.median(t1) / 1e9
     return {"value": round(byts / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "cpu_model": _cpu_model(), "single_thread_gbs": round(one, 3),
             "sample": (f"quantize+dequantize of the first 2^28 elements of the step's bf16 input "
                        f"({threads} threads over disjoint block ranges) and single-threaded "
-                       f"Q8_0/Q4_0 dequant of 2^18 blocks each; {dt:.2f} s wall")}
+                       f"Q8_0/Q4_0 dequant of 2^18 blocks each; {dt:.2f} s wall.  "
+                       f"single_thread_gbs: quantize+dequantize of 2^23 elements on one "
+                       f"thread, median of 3")}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def _pct(sorted_ts, f):
+    """Nearest-rank percentile of an already sorted list."""
+    return sorted_ts[min(len(sorted_ts) - 1, int(f * (len(sorted_ts) - 1) + 0.5))]
 
 
 # -------------------------------------------------------------------- ours --
@@ -369,8 +397,10 @@ def run_ours(args, rank, world, local):
     for k in names:
         ms = statistics.mean(per_kernel[k])
         gbs = byts[k] / (ms / 1e3) / 1e9
+        ts = sorted(per_kernel[k])
         kern[k] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
-                   "bytes": byts[k]}
+                   "bytes": byts[k], "median_ms": round(statistics.median(ts), 4),
+                   "p10_ms": round(_pct(ts, 0.1), 4), "p90_ms": round(_pct(ts, 0.9), 4)}
     # the dominant kernel: the one that takes the longest in the step
     dom = max(kern, key=lambda k: kern[k]["ms"])
     kname = {"quantize": "quantize_kernel<bf16,nf4,bs64>", "dequantize":
