@@ -20,9 +20,11 @@
 //  - 16-bit inputs: absmax from packed two-lane max of absolute values
 //    (NaN-propagating, so a block holding a NaN or inf is recognised by its
 //    absmax and takes the safe path);
-//  - xn by Markstein's correction from the block's reciprocal, two elements
-//    per instruction with the sm_100 fp32x2 FMA / MUL (no per-element range
-//    check: see div_fast);
+//  - xn two elements per instruction with the sm_100 fp32x2 FMA / MUL: for
+//    16-bit inputs one product with the trailing term of a two-term
+//    reciprocal and one FMA with its leading term (div_fast2_2term), for fp32
+//    inputs Markstein's correction from the rounded reciprocal (no
+//    per-element range check: see div_fast);
 //  - the code from a bucket table (bq_search.cuh): one packed bucket
 //    computation per pair, one 64-bit shared load and one compare per
 //    element (16-entry tables: each lane reads its own interleaved copy, so
@@ -180,7 +182,10 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
 #pragma unroll
   for (int i = 0; i < O::EPT / 2; ++i) {
     float q0, q1;
-    div_fast2(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
+    if constexpr (DT == kF32)
+      div_fast2(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
+    else
+      div_fast2_2term(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
     float b0 = q0, b1 = q1;
     if constexpr (E == 16)
       unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
@@ -314,7 +319,8 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
   if (fast)
-    encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP>(w, make_scale_fast(A), t_base, ow);
+    encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP>(
+        w, DT == kF32 ? make_scale_fast(A) : make_scale_fast_2term(A), t_base, ow);
   else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;

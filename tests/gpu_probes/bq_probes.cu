@@ -26,16 +26,18 @@ __device__ __forceinline__ bool same_quotient(float a, float b) {
   return __float_as_uint(a) == __float_as_uint(b) || (a == 0.0f && b == 0.0f);
 }
 
-// The quantize kernels' bucket path divides elements in pairs with the packed
-// Markstein form (div_fast2) for every block whose absmax is in [2^-60, 2^60],
-// without a per-element check: it needs the exact quotient, except that when
-// the exact quotient is below 2^-38 in magnitude the result only has to be
-// below 2^-38 too.  The safe path uses IEEE division for |x| < A 2^-40.
-// Both are checked; the packed form on both lanes (the second with -x).
+// The quantize kernels' bucket path divides elements in pairs for every block
+// whose absmax is in [2^-60, 2^60], without a per-element check: with the
+// packed Markstein form (div_fast2) for fp32 inputs and the packed two-term
+// form (div_fast2_2term) for 16-bit inputs.  It needs the exact quotient,
+// except that when the exact quotient is below 2^-38 in magnitude the result
+// only has to be below 2^-37.  The safe path uses IEEE division for |x| < A
+// 2^-40.  All are checked; the packed forms on both lanes (the second with -x).
 __device__ __forceinline__ bool bucket_path_ok(float got, float want) {
-  return same_quotient(got, want) || (fabsf(got) < 0x1p-38f && fabsf(want) < 0x1p-38f);
+  return same_quotient(got, want) || (fabsf(got) < 0x1p-37f && fabsf(want) < 0x1p-38f);
 }
 
+template <bool TWO_TERM>
 __device__ __forceinline__ bool division_ok(float x, float A) {
   const bq::BlockScale s = bq::make_scale(A);
   const float w0 = __fdiv_rn(x, A), w1 = __fdiv_rn(-x, A);
@@ -44,6 +46,10 @@ __device__ __forceinline__ bool division_ok(float x, float A) {
     float q0, q1;
     bq::div_fast2(x, -x, s, q0, q1);
     ok = bucket_path_ok(q0, w0) && bucket_path_ok(q1, w1);
+    if constexpr (TWO_TERM) {
+      bq::div_fast2_2term(x, -x, bq::make_scale_fast_2term(A), q0, q1);
+      ok = ok && bucket_path_ok(q0, w0) && bucket_path_ok(q1, w1);
+    }
   }
   const float safe = fabsf(x) < s.theta ? bq::div_exact(x, A) : bq::div_fast(x, s);
   return ok && same_quotient(safe, w0);
@@ -65,7 +71,7 @@ __global__ void div16_all(int a_lo) {
   for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
     const float x = bq::widen_pair_elem<DT>(xb, 0);
     if (!isfinite(x) || !(fabsf(x) <= A)) continue;
-    if (!division_ok(x, A)) report(xb, a_bits);
+    if (!division_ok<true>(x, A)) report(xb, a_bits);
   }
 }
 
@@ -90,7 +96,7 @@ __global__ void div32_random(uint64_t count, uint64_t seed) {
     float x = __uint_as_float(xb);
     if (!isfinite(A) || !isfinite(x) || A == 0.0f) continue;
     if (fabsf(x) > A) { const float t = A; A = fabsf(x); x = copysignf(t, x); }
-    if (!division_ok(x, A)) report(__float_as_uint(x), __float_as_uint(A));
+    if (!division_ok<false>(x, A)) report(__float_as_uint(x), __float_as_uint(A));
   }
 }
 
