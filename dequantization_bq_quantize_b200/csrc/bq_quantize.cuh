@@ -28,7 +28,8 @@
 //  - the code from a bucket table (bq_search.cuh): one packed bucket
 //    computation per pair, one 64-bit shared load and one compare per
 //    element (16-entry tables: each lane reads its own interleaved copy, so
-//    the loads never conflict on banks);
+//    the loads never conflict on banks); 256-entry tables whose codes step by
+//    one: one 32-bit shared load and one add per element (kModeLutI);
 //  - codes inserted into the output words with bit-field inserts.
 // Blocks whose absmax is outside [2^-60, 2^60] (or not finite), and codebooks
 // without a bucket table, take the safe path: IEEE division where Markstein's
@@ -93,6 +94,11 @@ __device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
   asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 
 template <int DT>
 __device__ __forceinline__ float tile_elem(const uint32_t (&w)[kThreadWords], int j) {
@@ -137,10 +143,21 @@ __device__ __forceinline__ uint32_t lut_addr(float b, uint32_t t_base) {
   }
 }
 
-template <int E>
+template <int E, int MODE>
 __device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut, int lane) {
   if constexpr (E == 16) return smem_u32(&lut.r[0][lane & 15]) - 128u * (0x4B400000u - 15u);
+  else if constexpr (MODE == kModeLutI) return smem_u32(lut.i) + 4u * 3073u;
   else return smem_u32(lut.e) + 8u * 1537u;
+}
+
+// kModeLutI (256-entry tables): i[bucket256i(q)] + key(q), whose byte 2 is
+// the code.  t_base = &i[3073]; the bucket offset (idx XOR sign mask) is
+// negative for negative q (32-bit wrap-around arithmetic).
+__device__ __forceinline__ uint32_t lut_int_sum(float q, uint32_t t_base) {
+  const uint32_t u = __float_as_uint(q);
+  const uint32_t g = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31);
+  const uint32_t idx = (max(u & 0x7fffffffu, 0x33800000u) - 0x33800000u) >> 16;
+  return lds_u32((idx ^ g) * 4u + t_base) + ((u ^ g) & 0xffffu);
 }
 
 // Weight of element j within its 16-bit half of the output: a half holds 4
@@ -166,6 +183,8 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 //             code * weight, every value an exact integer below 2^24; the
 //             first element of a half brings the 2^23), and the halves' low
 //             bytes are merged with one byte permute per word.
+//  kModeLutI (256-entry tables): code = byte 2 of i[b] + key(q)
+//             (bq_search.cuh); byte permutes gather four codes into a word.
 //  REMAP (16-entry tables like FP4, whose +-0 pair makes one step of two):
 //             the table holds ranks of the distinct values, which step by
 //             one; each nibble >= 8 then gets 1 added (ranks 8..14 -> codes
@@ -177,6 +196,7 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
   constexpr int NH = 2 * O::NW;                 // 16-bit halves
   constexpr int PER_HALF = O::EPT / NH;         // elements per half (4 or 2)
   float hacc[NH];
+  uint32_t pair[2 * O::NW];  // kModeLutI: codes of elements 2i, 2i+1 in bytes 0, 1
 #pragma unroll
   for (int k = 0; k < O::NW; ++k) ow[k] = 0u;
 #pragma unroll
@@ -186,6 +206,11 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
       div_fast2(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
     else
       div_fast2_2term(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
+    if constexpr (MODE == kModeLutI) {
+      static_assert(E == 256, "integer select is built for 256-entry tables only");
+      pair[i] = __byte_perm(lut_int_sum(q0, t_base), lut_int_sum(q1, t_base), 0x0062);
+      continue;
+    }
     float b0 = q0, b1 = q1;
     if constexpr (E == 16)
       unpack2(fma2(pack2(q0, q1), pack2(15.0f, 15.0f), pack2(12582912.0f, 12582912.0f)), b0, b1);
@@ -208,6 +233,10 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
       ow[j0 / O::PER_WORD] = bfi(c0, ow[j0 / O::PER_WORD], code_pos<E>(j0), O::L);
       ow[j1 / O::PER_WORD] = bfi(c1, ow[j1 / O::PER_WORD], code_pos<E>(j1), O::L);
     }
+  }
+  if constexpr (MODE == kModeLutI) {
+#pragma unroll
+    for (int k = 0; k < O::NW; ++k) ow[k] = __byte_perm(pair[2 * k], pair[2 * k + 1], 0x5410);
   }
   if constexpr (MODE == kModeLutF) {
 #pragma unroll
@@ -316,7 +345,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   uint32_t ow[O::NW];
   // bucket path: the block's reciprocal is valid for Markstein's form (the
   // per-element condition is not needed, see div_fast); NaN fails both tests
-  constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF;
+  constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF || MODE == kModeLutI;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
   if (fast)
     encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP>(
@@ -366,7 +395,7 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 template <int DT, int E, int TPB, int MODE, bool REMAP = false>
 __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int ct) {
   constexpr int BPT = kQConsumers / TPB;
-  const uint32_t t_base = lut_base<E>(s.lut, ct & 31);
+  const uint32_t t_base = lut_base<E, MODE>(s.lut, ct & 31);
   const uint32_t ntiles = static_cast<uint32_t>(p.full_tiles);  // < 2^24 (host check)
   uint32_t iter = 0;
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
@@ -439,6 +468,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
   if (mode == kModeLutF && E == 16 && s.tab.remap8)
     consumer_main<DT, E, TPB, kModeLutF, E == 16>(s, p, ct);
   else if (mode == kModeLutF) consumer_main<DT, E, TPB, kModeLutF>(s, p, ct);
+  else if (E == 256 && mode == kModeLutI) consumer_main<DT, E, TPB, E == 256 ? kModeLutI : kModeLutF>(s, p, ct);
   else if (mode == kModeLut) consumer_main<DT, E, TPB, kModeLut>(s, p, ct);
   else if (mode == kModeBsearch) consumer_main<DT, E, TPB, kModeBsearch>(s, p, ct);
   else consumer_main<DT, E, TPB, kModeScan>(s, p, ct);

@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(256) search_all(const float* code, int* mode_o
     const float xn = __uint_as_float(bits);
     uint32_t got;
     if (mode == bq::kModeLutF) got = bq::search<E, bq::kModeLutF>(xn, s.tab, s.lut);
+    else if (mode == bq::kModeLutI)
+      got = bq::search<E, E == 256 ? bq::kModeLutI : bq::kModeLutF>(xn, s.tab, s.lut);
     else if (mode == bq::kModeLut) got = bq::search<E, bq::kModeLut>(xn, s.tab, s.lut);
     else if (mode == bq::kModeBsearch) got = bq::search<E, bq::kModeBsearch>(xn, s.tab, s.lut);
     else got = bq::search<E, bq::kModeScan>(xn, s.tab, s.lut);
@@ -150,15 +152,18 @@ __global__ void __launch_bounds__(256) search_all(const float* code, int* mode_o
 
 template <int E, int MODE>
 __global__ void __launch_bounds__(256) search_forced(const float* code, int* mode_out) {
-  // same sweep, but with a forced search form (to test the bisection form too)
+  // same sweep, but with a forced search form: the bisection form (built for
+  // every valid table), or the float-select form of a 256-entry table that
+  // would otherwise get the integer form (built with that form disallowed)
   extern __shared__ uint8_t raw[];
   ProbeSmem<E>& s = *reinterpret_cast<ProbeSmem<E>*>(raw);
   const int ct = threadIdx.x;
-  bq::build_search<E, 256>(s.tab, s.lut, code, ct);
+  bq::build_search<E, 256>(s.tab, s.lut, code, ct, MODE != bq::kModeLutF);
   if (ct < E) s.c[ct] = code[ct];
   __syncthreads();
   if (blockIdx.x == 0 && ct == 0) *mode_out = s.tab.mode;
   if (s.tab.mode == bq::kModeScan) return;   // forced forms need a valid table
+  if (MODE == bq::kModeLutF && s.tab.mode != bq::kModeLutF) return;  // reported via mode_out
   const uint64_t npos = 0x3f800001ull;
   const uint64_t total = 2 * npos;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -263,7 +268,8 @@ __attribute__((visibility("default"))) int probe_div32(unsigned long long count,
   return finish(mm, fa, fb);
 }
 
-// mode_request: -1 = whatever the builder picks, 1 = force the bisection form.
+// mode_request: -1 = whatever the builder picks, 1 = force the bisection form,
+// 3 = the float-select form of a 256-entry table (integer form disallowed).
 __attribute__((visibility("default"))) int probe_search(const float* code, int entries,
                                                         int mode_request, int* mode_out,
                                                         unsigned long long* mm, unsigned int* fa,
@@ -275,6 +281,8 @@ __attribute__((visibility("default"))) int probe_search(const float* code, int e
   }
   if (mode_request == 1)
     return run_search<256>(search_forced<256, bq::kModeBsearch>, code, mode_out, mm, fa, fb);
+  if (mode_request == 3)
+    return run_search<256>(search_forced<256, bq::kModeLutF>, code, mode_out, mm, fa, fb);
   return run_search<256>(search_all<256>, code, mode_out, mm, fa, fb);
 }
 

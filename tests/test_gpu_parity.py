@@ -477,14 +477,15 @@ def test_division_fp32_random(probes):
 
 # search forms: 0 = bucket table, integer select; 3 = bucket table, float
 # select (codes step by one at every threshold; FP4's +-0 pair, the one step
-# of two, is handled by selecting over ranks and adding 1 from rank 8 on).
-# "dup34" repeats entries 3 and 4, a step of two that only the integer
-# select handles.
+# of two, is handled by selecting over ranks and adding 1 from rank 8 on);
+# 4 = 256-entry tables: 4-byte entries over finer buckets, select on the
+# float bits.  "dup34" repeats entries 3 and 4, a step of two that only the
+# integer select handles.
 _DUP34 = TABLES["nf4"].copy()
 _DUP34[4] = _DUP34[3]
 
 
-@pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 3), ("dyn8", 3),
+@pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 3), ("dyn8", 4),
                                               ("dup34", 0)])
 @pytest.mark.parametrize("force", [-1, 1], ids=["chosen", "bisection"])
 def test_search_exhaustive(probes, name, expect_mode, force):
@@ -495,6 +496,19 @@ def test_search_exhaustive(probes, name, expect_mode, force):
     assert probes.probe_search(code.data_ptr(), table.size, force, ctypes.byref(mode),
                                ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
     assert mode.value == expect_mode
+    assert mm.value == 0, f"{mm.value} mismatches, first xn bits {fa.value:#x} got|want {fb.value:#x}"
+
+
+def test_search_exhaustive_dyn8_float_select(probes):
+    """The float-select form of a 256-entry table, which dyn8 no longer gets
+    by default, checked over every float in [-1, 1] too."""
+    table = TABLES["dyn8"]
+    code = code_dev(table)
+    mode = ctypes.c_int(-1)
+    mm, fa, fb = _outs()
+    assert probes.probe_search(code.data_ptr(), table.size, 3, ctypes.byref(mode),
+                               ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
+    assert mode.value == 3
     assert mm.value == 0, f"{mm.value} mismatches, first xn bits {fa.value:#x} got|want {fb.value:#x}"
 
 
