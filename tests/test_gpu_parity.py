@@ -483,13 +483,21 @@ def test_division_fp32_random(probes):
 # integer select handles.
 _DUP34 = TABLES["nf4"].copy()
 _DUP34[4] = _DUP34[3]
+# dyn8 with its codes -5.5e-7, 0, 5.5e-7 replaced by -1e-6, -2.5e-7, 2.9e-7:
+# every gap still exceeds 2 ulp(1 + max|c|), but the threshold between the
+# last two (about 2e-8) falls in the fine bucket around zero, so the 4-byte
+# form is refused and the float select is built
+_DYN8TINY = TABLES["dyn8"].copy()
+_k0 = int(np.nonzero(_DYN8TINY == 0)[0][0])
+_DYN8TINY[_k0 - 1:_k0 + 2] = np.array([-1.0e-6, -2.5e-7, 2.9e-7], np.float32)
+_NAMED = {"dup34": _DUP34, "dyn8tiny": _DYN8TINY}
 
 
 @pytest.mark.parametrize("name,expect_mode", [("nf4", 3), ("fp4", 3), ("dyn8", 4),
-                                              ("dup34", 0)])
+                                              ("dup34", 0), ("dyn8tiny", 3)])
 @pytest.mark.parametrize("force", [-1, 1], ids=["chosen", "bisection"])
 def test_search_exhaustive(probes, name, expect_mode, force):
-    table = _DUP34 if name == "dup34" else TABLES[name]
+    table = _NAMED.get(name, TABLES.get(name))
     code = code_dev(table)
     mode = ctypes.c_int(-1)
     mm, fa, fb = _outs()
@@ -510,6 +518,24 @@ def test_search_exhaustive_dyn8_float_select(probes):
                                ctypes.byref(mm), ctypes.byref(fa), ctypes.byref(fb)) == 0
     assert mode.value == 3
     assert mm.value == 0, f"{mm.value} mismatches, first xn bits {fa.value:#x} got|want {fb.value:#x}"
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_256_entry_float_select_in_kernel(dtype):
+    """The quantize kernel on a 256-entry table that gets the float select
+    (the dyn8 variant above): codes, absmax and dequantized values equal the
+    oracle's; tiles, tail blocks and an all-zero block included."""
+    n, bs = 3 * 8192 + 333, 64
+    x = small_input(n, dtype, bs, seed=31)
+    table = _DYN8TINY
+    ga, go, _ = gpu_quantize(x, dtype, bs, table)
+    oa, oo = oracle.quantize_blockwise(x, dtype, bs, table)
+    assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32))
+    assert np.array_equal(go, oo)
+    gy = gpu_dequantize(oo, oa, n, bs, table, dtype)
+    oy = oracle.dequantize_blockwise(oo, oa, n, bs, table, dtype)
+    assert np.array_equal(gy.view(np.uint32 if dtype == "f32" else np.uint16),
+                          oy.view(np.uint32 if dtype == "f32" else np.uint16))
 
 
 def test_bounded_wait_gives_up_and_context_survives(probes):
