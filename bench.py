@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
+    ap.add_argument("--codebook", choices=["nf4", "fp4", "dyn8"], default="nf4",
+                    help="table of the step's quantize / dequantize (profiling aid; the benchmark "
+                         "line is nf4; other tables need --no-e2e)")
     ap.add_argument("--gguf-kinds", default="",
                     help="gguf workload: comma-separated types to run (e.g. q4_k,q8_0_encode)")
     ap.add_argument("--gguf-sizes", default="small,matrix",
@@ -62,18 +65,21 @@ def parse_args():
 
 # ------------------------------------------------------------------ bytes --
 
-def quant_bytes(n, bs, elem=2):
+def quant_bytes(n, bs, elem=2, entries=16):
     """Algorithmic bytes of one quantize (or dequantize) launch: n*elem input
-    (output), ceil(n/2) packed codes, 4 bytes of absmax per block."""
-    return n * elem + (n + 1) // 2 + 4 * ((n + bs - 1) // bs)
+    (output), ceil(n/2) packed 4-bit codes (n 8-bit codes for 256-entry
+    tables), 4 bytes of absmax per block."""
+    codes = (n + 1) // 2 if entries == 16 else n
+    return n * elem + codes + 4 * ((n + bs - 1) // bs)
 
 
 def gguf_bytes(nblk, block_bytes, out_elem=2):
     return nblk * block_bytes + 32 * nblk * out_elem
 
 
-def step_bytes(n, nblk, only="all"):
-    parts = {"quantize": quant_bytes(n, BS), "dequantize": quant_bytes(n, BS),
+def step_bytes(n, nblk, only="all", entries=16):
+    parts = {"quantize": quant_bytes(n, BS, entries=entries),
+             "dequantize": quant_bytes(n, BS, entries=entries),
              "q8_0": gguf_bytes(nblk, 34), "q4_0": gguf_bytes(nblk, 18)}
     if only != "all":
         return {only: parts[only]}
@@ -303,7 +309,7 @@ def _pct(sorted_ts, f):
 # -------------------------------------------------------------------- ours --
 
 class Workload:
-    def __init__(self, n, rank, device):
+    def __init__(self, n, rank, device, codebook="nf4"):
         import dequantization_bq_quantize_b200 as bq
         self.bq = bq
         bq.lib()
@@ -313,9 +319,12 @@ class Workload:
         x_cpu, self.outliers = synth.large_outliers(n=n, seed=3 + 1000 * rank)
         self.x_cpu = x_cpu
         self.x = x_cpu.to(device)
-        self.code = torch.from_numpy(codebooks.nf4()).to(device)
+        self.codebook = codebook
+        self.code = torch.from_numpy(codebooks.get(codebook)).to(device)
+        self.entries = self.code.numel()
         self.absmax = torch.empty(self.nb, dtype=torch.float32, device=device)
-        self.q = torch.empty((n + 1) // 2, dtype=torch.uint8, device=device)
+        self.q = torch.empty((n + 1) // 2 if self.entries == 16 else n, dtype=torch.uint8,
+                             device=device)
         self.y = torch.empty(n, dtype=torch.bfloat16, device=device)
         q8 = synth.gguf_blocks(self.nblk, "q8_0", seed=4 + 1000 * rank)
         q4 = synth.gguf_blocks(self.nblk, "q4_0", seed=5 + 1000 * rank)
@@ -335,11 +344,11 @@ class Workload:
         bq = self.bq
         if name == "quantize":
             st = bq.bq_quantize_blockwise(self.x.data_ptr(), bq.BQ_BF16, self.n, BS,
-                                          self.code.data_ptr(), 16, self.absmax.data_ptr(),
+                                          self.code.data_ptr(), self.entries, self.absmax.data_ptr(),
                                           self.q.data_ptr(), stream)
         elif name == "dequantize":
             st = bq.bq_dequantize_blockwise(self.q.data_ptr(), self.absmax.data_ptr(), self.n, BS,
-                                            self.code.data_ptr(), 16, self.y.data_ptr(),
+                                            self.code.data_ptr(), self.entries, self.y.data_ptr(),
                                             bq.BQ_BF16, stream)
         elif name == "q8_0":
             st = bq.bq_dequant_q8_0(self.q8.data_ptr(), self.nblk, self.y8.data_ptr(), bq.BQ_BF16,
@@ -353,11 +362,13 @@ class Workload:
 
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = Workload(args.n, rank, dev)
+    if args.codebook != "nf4" and not args.no_e2e:
+        raise SystemExit("--codebook other than nf4 needs --no-e2e")
+    w = Workload(args.n, rank, dev, args.codebook)
     names = w.kernels(args.only)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
-    byts = step_bytes(w.n, w.nblk, args.only)
+    byts = step_bytes(w.n, w.nblk, args.only, w.entries)
     step_total = sum(byts.values())
 
     for _ in range(args.warmup):
@@ -403,9 +414,11 @@ def run_ours(args, rank, world, local):
                    "p10_ms": round(_pct(ts, 0.1), 4), "p90_ms": round(_pct(ts, 0.9), 4)}
     # the dominant kernel: the one that takes the longest in the step
     dom = max(kern, key=lambda k: kern[k]["ms"])
-    kname = {"quantize": "quantize_kernel<bf16,nf4,bs64>", "dequantize":
-             "dequant_stream_kernel<nf4,bf16>", "q8_0": "gguf_kernel<q8_0,bf16>",
-             "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
+    cb = w.codebook
+    kname = {"quantize": f"quantize_kernel<bf16,{cb},bs64>",
+             "dequantize": (f"dequant_stream_kernel<{cb},bf16>" if w.entries == 16
+                            else f"dequant_kernel<{cb},bf16>"),
+             "q8_0": "gguf_kernel<q8_0,bf16>", "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
     roof = {"bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak, "unit": "GB/s",
             "frac": kern[dom]["frac"], "traffic": recorded_traffic(kname),
             "kernel": kname, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"}
@@ -420,7 +433,8 @@ def run_ours(args, rank, world, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "n": w.n, "blocksize": BS, "codebook": "nf4",
+            "config": {"workload": WORKLOAD.replace("NF4", w.codebook.upper()), "n": w.n,
+                       "blocksize": BS, "codebook": w.codebook,
                        "gguf_blocks": w.nblk, "outliers": w.outliers, "kernels": names,
                        "l2": "inputs larger than L2 (126 MB); no flush",
                        "parallelism": f"dp{world} (independent shards, no collective)"},
