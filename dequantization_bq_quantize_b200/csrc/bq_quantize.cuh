@@ -151,13 +151,13 @@ __device__ __forceinline__ uint32_t lut_base(const Lut<E>& lut, int lane) {
 }
 
 // kModeLutI (256-entry tables): i[bucket256i(q)] + key(q), whose byte 2 is
-// the code.  t_base = &i[3073]; the bucket offset (idx XOR sign mask) is
-// negative for negative q (32-bit wrap-around arithmetic).
+// the code.  t_base = &i[3073]; the bucket offset is negative for negative q
+// (32-bit wrap-around arithmetic).
 __device__ __forceinline__ uint32_t lut_int_sum(float q, uint32_t t_base) {
-  const uint32_t u = __float_as_uint(q);
-  const uint32_t g = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31);
-  const uint32_t idx = (max(u & 0x7fffffffu, 0x33800000u) - 0x33800000u) >> 16;
-  return lds_u32((idx ^ g) * 4u + t_base) + ((u ^ g) & 0xffffu);
+  int32_t off;
+  uint32_t key;
+  lut_int_index(q, off, key);
+  return lds_u32(static_cast<uint32_t>(off) * 4u + t_base) + key;
 }
 
 // Weight of element j within its 16-bit half of the output: a half holds 4
