@@ -361,9 +361,9 @@ class Workload:
 
 
 def run_ours(args, rank, world, local):
-    dev = torch.device("cuda", torch.cuda.current_device())
     if args.codebook != "nf4" and not args.no_e2e:
         raise SystemExit("--codebook other than nf4 needs --no-e2e")
+    dev = torch.device("cuda", torch.cuda.current_device())
     w = Workload(args.n, rank, dev, args.codebook)
     names = w.kernels(args.only)
     stream = torch.cuda.current_stream()

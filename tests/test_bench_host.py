@@ -1,0 +1,75 @@
+"""Host-side checks of bench.py: the algorithmic byte counts behind every GB/s
+and roofline figure, the percentile helper, and the JSON line of the
+reference arm (the oracle timed on the host cores), run on the CPU."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_quantize_bytes_match_the_per_element_figures():
+    # in + out per element: s + 1/2 + 4/bs for 4-bit codes, s + 1 + 4/bs for
+    # 8-bit codes; the 1 GiB bf16 NF4 bs 64 case moves 2^30 + 2^28 + 2^25 bytes
+    n = 1 << 29
+    assert bench.quant_bytes(n, 64) == (1 << 30) + (1 << 28) + (1 << 25) == 1_375_731_712
+    assert bench.quant_bytes(n, 64, entries=256) == (1 << 30) + (1 << 29) + (1 << 25)
+    assert bench.quant_bytes(n, 64, elem=4) == (1 << 31) + (1 << 28) + (1 << 25)
+    # odd n: the last packed byte is shared, the tail block has its own absmax
+    assert bench.quant_bytes(8388645, 64) == 2 * 8388645 + 4194323 + 4 * 131073
+
+
+def test_gguf_bytes_match_the_block_formats():
+    nblk = 4096 * 14336 // 32
+    assert bench.gguf_bytes(nblk, 34) == 62_390_272 + 117_440_512   # Q8_0 -> bf16
+    assert bench.gguf_bytes(nblk, 18) == 33_030_144 + 117_440_512   # Q4_0 -> bf16
+    parts = bench.step_bytes(1 << 29, nblk)
+    assert set(parts) == {"quantize", "dequantize", "q8_0", "q4_0"}
+    assert parts["quantize"] == parts["dequantize"] == 1_375_731_712
+    assert bench.step_bytes(1 << 29, nblk, "q4_0") == {"q4_0": 150_470_656}
+
+
+def test_percentiles():
+    ts = sorted([5.0, 1.0, 4.0, 2.0, 3.0, 9.0, 7.0, 8.0, 6.0, 10.0, 11.0])
+    assert bench._pct(ts, 0.0) == 1.0
+    assert bench._pct(ts, 0.5) == 6.0
+    assert bench._pct(ts, 1.0) == 11.0
+    assert bench._pct([3.0], 0.9) == 3.0
+
+
+def test_reference_arm_json_line():
+    """`--impl reference` times the oracle on the host and prints one line
+    with the same metric and unit as the GPU arm, its e2e object and its
+    cpu_baseline object."""
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    with open(os.path.join(ROOT, "BASELINE.json")) as f:
+        metric = json.load(f)["metric"]
+    assert d["impl"] == "reference" and d["metric"] == metric and d["unit"] == "GB/s"
+    assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 1
+    assert d["value"] > 0
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert cb["sample"]
+
+
+def test_codebook_option_needs_no_e2e(monkeypatch):
+    """The end-to-end path is NF4-only; other tables must be asked for with
+    --no-e2e (checked before any device work)."""
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--codebook", "dyn8"])
+    args = bench.parse_args()
+    assert args.codebook == "dyn8" and not args.no_e2e
+    with pytest.raises(SystemExit):
+        bench.run_ours(args, 0, 1, 0)
