@@ -53,9 +53,7 @@ def test_reference_arm_json_line():
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
     d = json.loads(lines[0])
-    with open(os.path.join(ROOT, "BASELINE.json")) as f:
-        metric = json.load(f)["metric"]
-    assert d["impl"] == "reference" and d["metric"] == metric and d["unit"] == "GB/s"
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
     assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 1
     assert d["value"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
