@@ -40,6 +40,8 @@
 // byte.
 #pragma once
 
+#include <type_traits>
+
 #include "bq_common.cuh"
 
 namespace bq {
@@ -93,6 +95,34 @@ __device__ __forceinline__ void load8_at2(const uint8_t* ptr, uint32_t& w0, uint
   w1 = __funnelshift_r(x1, x2, sh);
 }
 
+// Eight bytes at a shared address whose remainder mod 8 is BA, known at
+// compile time (BA = -1: unknown, any 2-byte aligned address).  K-quant
+// super-blocks sit at u * BB bytes of an 8-byte aligned staging buffer and
+// are read at multiples of 8 inside the block, so pass u of a warp step reads
+// at remainder (u * BB) mod 8: one 64-bit load, two 32-bit loads, or three and
+// a fixed 16-bit funnel shift (Q3_K's 110- and Q6_K's 210-byte blocks
+// alternate).
+template <int BA>
+__device__ __forceinline__ void load8(const uint8_t* ptr, uint32_t& w0, uint32_t& w1) {
+  if constexpr (BA < 0) {
+    load8_at2(ptr, w0, w1);
+  } else if constexpr (BA == 0) {
+    const uint2 q = *reinterpret_cast<const uint2*>(ptr);
+    w0 = q.x;
+    w1 = q.y;
+  } else if constexpr (BA == 4) {
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(ptr);
+    w0 = wp[0];
+    w1 = wp[1];
+  } else {
+    static_assert(BA == 2 || BA == 6, "2-byte aligned reads only");
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(ptr - 2);
+    const uint32_t x0 = wp[0], x1 = wp[1], x2 = wp[2];
+    w0 = __funnelshift_r(x0, x1, 16);
+    w1 = __funnelshift_r(x1, x2, 16);
+  }
+}
+
 __device__ __forceinline__ float half_at(const uint8_t* p) {
   return __half2float(*reinterpret_cast<const __half*>(p));
 }
@@ -126,7 +156,8 @@ __device__ __forceinline__ void bytes_to_values(uint32_t w0, uint32_t w1, float 
 }
 
 // Decode outputs 8*part .. 8*part+7 of the block at bp (part < EPB / 8).
-template <int KIND>
+// BA: bp's remainder mod 8 when known at compile time, else -1.
+template <int KIND, int BA = -1>
 __device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float (&v)[8]) {
   using T = GTraits<KIND>;
   uint32_t w0, w1;
@@ -191,7 +222,7 @@ __device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float 
     const uint32_t scb = bp[part >> 1];
     const float a = half_at(bp + 80) * static_cast<float>(scb & 15u);  // exact
     const float b = half_at(bp + 82) * static_cast<float>(scb >> 4);   // exact
-    load8_at2(bp + 16 + 32 * n + 16 * hh + s8, w0, w1);
+    load8<BA>(bp + 16 + 32 * n + 16 * hh + s8, w0, w1);
     w0 = (w0 >> (2 * c)) & 0x03030303u;
     w1 = (w1 >> (2 * c)) & 0x03030303u;
     bytes_to_values<true>(w0, w1, 8388608.0f, a, -b, v);
@@ -205,8 +236,8 @@ __device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float 
     const int scale = static_cast<int>(lo4 | (hi2 << 4)) - 32;
     const float a = half_at(bp + 108) * static_cast<float>(scale);  // exact
     uint32_t m0, m1;
-    load8_at2(bp + 32 + 32 * n + 16 * hh + s8, w0, w1);
-    load8_at2(bp + 16 * hh + s8, m0, m1);
+    load8<BA>(bp + 32 + 32 * n + 16 * hh + s8, w0, w1);
+    load8<BA>(bp + 16 * hh + s8, m0, m1);
     const int hs = 4 * n + c;
     w0 = ((w0 >> (2 * c)) & 0x03030303u) | (((m0 >> hs) & 0x01010101u) << 2);
     w1 = ((w1 >> (2 * c)) & 0x03030303u) | (((m1 >> hs) & 0x01010101u) << 2);
@@ -215,8 +246,8 @@ __device__ __forceinline__ void gguf_decode8(const uint8_t* bp, int part, float 
     // part = 16n + 4c + r: half n, 32-element chunk c, outputs 8r..8r+7 of it
     const int n = part >> 4, c = (part >> 2) & 3, r = part & 3;
     uint32_t h0, h1;
-    load8_at2(bp + 64 * n + 32 * (c & 1) + 8 * r, w0, w1);
-    load8_at2(bp + 128 + 32 * n + 8 * r, h0, h1);
+    load8<BA>(bp + 64 * n + 32 * (c & 1) + 8 * r, w0, w1);
+    load8<BA>(bp + 128 + 32 * n + 8 * r, h0, h1);
     const int sl = 4 * (c >> 1), sh = 2 * c;
     w0 = ((w0 >> sl) & 0x0F0F0F0Fu) | (((h0 >> sh) & 0x03030303u) << 4);
     w1 = ((w1 >> sl) & 0x0F0F0F0Fu) | (((h1 >> sh) & 0x03030303u) << 4);
@@ -246,6 +277,15 @@ __device__ __forceinline__ void store8(void* y, int64_t e0, const float (&v)[8],
   }
 }
 
+// f(integral_constant<int, U>) for U = B .. E-1, in order
+template <int B, int E, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (B < E) {
+    f(std::integral_constant<int, B>{});
+    static_for<B + 1, E>(f);
+  }
+}
+
 template <int KIND, int OT>
 __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
   using T = GTraits<KIND>;
@@ -259,7 +299,7 @@ __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
   constexpr int LOADS = (STEP_CHUNKS + 31) / 32;   // per lane: 2 to 4
   static_assert(STEP_BYTES % 16 == 0, "a step must be whole 16-byte chunks");
   // 16 bytes of padding: the 8-byte reads of the last block may load one
-  // aligned word past the block
+  // aligned word past the block.  Every warp's buffer starts 16-byte aligned.
   __shared__ __align__(16) uint8_t buf[kGThreads / 32][STEP_BYTES + 16];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -302,15 +342,17 @@ __global__ void __launch_bounds__(kGThreads) gguf_kernel(const GParams p) {
     __syncwarp();
 
     const int part = lane % LPB;
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
+    // one pass per u; with one block per pass (K-quants) its offset u * BB,
+    // and so the alignment of its reads, is a compile-time constant
+    static_for<0, UNROLL>([&](auto uc) {
+      constexpr int u = decltype(uc)::value;
       const int bl = u * GROUP + lane / LPB;
       if (bl < nblk) {
         float v[8];
-        gguf_decode8<KIND>(wb + bl * BB, part, v);
+        gguf_decode8<KIND, GROUP == 1 ? (u * BB) % 8 : -1>(wb + bl * BB, part, v);
         store8<OT>(p.y, (blk0 + bl) * T::EPB + part * 8, v, p.vec != 0);
       }
-    }
+    });
     __syncwarp();
   }
 }
