@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libbq.so")
 
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_CUDA = 0, 1, 2, 3
 BQ_F32, BQ_F16, BQ_BF16 = 0, 1, 2
+BQ_NOALLOC_MAX_BLOCKS = 1 << 20  # bq_quantize_blockwise_nested_noalloc's limit
 
 # GGUF block types: (outputs per block, bytes per block)
 # ("bf16": plain bfloat16 values, one per 2-byte "block")
@@ -32,7 +33,8 @@ GGUF_ENCODERS = ("q8_0", "q4_0")
 
 EXPORTED = (
     "bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_quantize_blockwise_nested",
-    "bq_dequantize_blockwise_nested", "bq_quantize_blockwise_host",
+    "bq_quantize_blockwise_nested_noalloc", "bq_dequantize_blockwise_nested",
+    "bq_quantize_blockwise_host",
 ) + tuple("bq_dequant_" + k for k in GGUF_TYPES) + tuple(
     "bq_quantize_" + k for k in GGUF_ENCODERS) + (
     "bq_status_string", "bq_last_cuda_error", "bq_device_fault", "bq_abi_version",
@@ -69,13 +71,15 @@ def lib():
             getattr(L, "bq_quantize_" + k).restype = ctypes.c_int
         L.bq_quantize_blockwise_nested.argtypes = [vp, i32, i64, i32, vp, i32, vp, i32, i32, vp,
                                                    vp, vp, vp, vp]
+        L.bq_quantize_blockwise_nested_noalloc.argtypes = [vp, i32, i64, i32, vp, i32, vp, i32,
+                                                           i32, vp, vp, vp, vp]
         L.bq_dequantize_blockwise_nested.argtypes = [vp, vp, vp, i64, i32, vp, i32, vp, i32, i32,
                                                      vp, i32, vp]
         L.bq_quantize_blockwise_host.argtypes = [vp, i32, i64, i32, vp, i32, vp, i32, i32, vp, vp,
                                                  vp, vp, vp, i64, i64, vp, vp]
         for f in ("bq_quantize_blockwise", "bq_dequantize_blockwise", "bq_device_fault",
                   "bq_quantize_blockwise_nested", "bq_dequantize_blockwise_nested",
-                  "bq_quantize_blockwise_host"):
+                  "bq_quantize_blockwise_nested_noalloc", "bq_quantize_blockwise_host"):
             getattr(L, f).restype = ctypes.c_int
         L.bq_status_string.argtypes = [ctypes.c_int]
         L.bq_status_string.restype = ctypes.c_char_p
@@ -111,6 +115,14 @@ def bq_quantize_blockwise_nested(x, x_dtype, n, blocksize, code, code_entries, c
     return lib().bq_quantize_blockwise_nested(x, x_dtype, n, blocksize, code, code_entries, code2,
                                               code2_entries, blocksize2, absmax, out, absmax2,
                                               qabsmax, stream)
+
+
+def bq_quantize_blockwise_nested_noalloc(x, x_dtype, n, blocksize, code, code_entries, code2,
+                                         code2_entries, blocksize2, out, absmax2, qabsmax,
+                                         stream):
+    return lib().bq_quantize_blockwise_nested_noalloc(x, x_dtype, n, blocksize, code,
+                                                      code_entries, code2, code2_entries,
+                                                      blocksize2, out, absmax2, qabsmax, stream)
 
 
 def bq_dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code, code_entries, code2,

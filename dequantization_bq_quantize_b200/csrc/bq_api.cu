@@ -365,6 +365,41 @@ bq_status gguf_encode_entry(const void* x, bq_dtype x_dtype, int64_t n, void* bl
 
 }  // namespace
 
+// ------------------------------------------ allocation-free nested quantize ---
+
+// First-level fp32 statistics of bq_quantize_blockwise_nested_noalloc: one
+// array per device, held from the library's load on that device until the
+// process exits, shared by every call (see include/bq.h).  Host code must not
+// pass this name to a kernel: on the host it is a stand-in object, not the
+// device address, which noalloc_stats() looks up.
+static __device__ __align__(256) float g_noalloc_stats[BQ_NOALLOC_MAX_BLOCKS];
+
+namespace {
+
+std::once_flag g_noalloc_once[kMaxDevices];
+float* g_noalloc_ptr[kMaxDevices] = {};
+cudaError_t g_noalloc_err[kMaxDevices] = {};
+
+// Device address of g_noalloc_stats on `dev`, looked up once per device with
+// that device current (the caller's current device).
+bq_status noalloc_stats(int dev, float** ptr) {
+  std::call_once(g_noalloc_once[dev], [&] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_stats);
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  });
+  if (g_noalloc_err[dev] != cudaSuccess)
+    return cuda_fail(g_noalloc_err[dev], "looking up the static statistics array");
+  if (!g_noalloc_ptr[dev]) {
+    t_err = "static statistics array has no device address";
+    return BQ_ERR_CUDA;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return BQ_OK;
+}
+
+}  // namespace
+
 // ===================================================================== ABI ==
 
 extern "C" {
@@ -463,6 +498,36 @@ bq_status bq_quantize_blockwise_nested(const void* x, bq_dtype x_dtype, int64_t 
   const int64_t nb = (n + blocksize - 1) / blocksize;
   return bq_quantize_blockwise(absmax, BQ_F32, nb, blocksize2, code2, code2_entries, absmax2,
                                qabsmax, stream);
+}
+
+bq_status bq_quantize_blockwise_nested_noalloc(const void* x, bq_dtype x_dtype, int64_t n,
+                                               int32_t blocksize, const float* code,
+                                               int32_t code_entries, const float* code2,
+                                               int32_t code2_entries, int32_t blocksize2,
+                                               uint8_t* out, float* absmax2, uint8_t* qabsmax,
+                                               cudaStream_t stream) {
+  t_err.clear();
+  if (n < 0 || !valid_dtype(x_dtype) || !valid_blocksize(blocksize) ||
+      !valid_blocksize(blocksize2) || (code_entries != 16 && code_entries != 256) ||
+      code2_entries != 256)
+    return BQ_ERR_INVALID_ARG;
+  if (n == 0) return BQ_OK;
+  const int64_t nb = (n + blocksize - 1) / blocksize;
+  if (nb > BQ_NOALLOC_MAX_BLOCKS) {
+    t_err = "n / blocksize exceeds BQ_NOALLOC_MAX_BLOCKS (2^20 blocks): use "
+            "bq_quantize_blockwise_nested with a caller-allocated absmax buffer";
+    return BQ_ERR_INVALID_ARG;
+  }
+  int dev;
+  DevInfo info;
+  bq_status s = current_device(&dev, &info);
+  if (s != BQ_OK) return s;
+  float* stats = nullptr;
+  s = noalloc_stats(dev, &stats);
+  if (s != BQ_OK) return s;
+  return bq_quantize_blockwise_nested(x, x_dtype, n, blocksize, code, code_entries, code2,
+                                      code2_entries, blocksize2, stats, out, absmax2, qabsmax,
+                                      stream);
 }
 
 bq_status bq_dequantize_blockwise_nested(const uint8_t* q, const uint8_t* qabsmax,

@@ -135,6 +135,48 @@ BQ_API bq_status bq_quantize_blockwise_nested(const void *x, bq_dtype x_dtype, i
                                   uint8_t *qabsmax, cudaStream_t stream);
 
 /*
+ * bq_quantize_blockwise_nested for callers that cannot allocate device
+ * memory.  (The source pages have no counterpart of this entry point; it
+ * exists for the way this library is embedded.)  Some callers cannot call
+ * cudaMalloc: for example a plug-in inside a host framework that owns all
+ * device memory (a caching allocator, or an arena planned before the run)
+ * and hands the plug-in only its inputs and outputs, where an allocation
+ * behind the framework's back would break its memory budget and can
+ * synchronize the device.  Such a caller usually wants only the compressed
+ * statistics, not the fp32 first-level statistics that
+ * bq_quantize_blockwise_nested writes to a caller buffer between its two
+ * launches.  This entry point keeps that intermediate array in a fixed
+ * device array inside the library instead, and otherwise behaves exactly
+ * like bq_quantize_blockwise_nested (same arguments without `absmax`, same
+ * outputs, bit for bit).
+ *
+ *  - Size limit: ceil(n / blocksize) <= BQ_NOALLOC_MAX_BLOCKS (2^20 blocks,
+ *    4 MiB of fp32), i.e. n <= 2^20 * blocksize.  Larger inputs return
+ *    BQ_ERR_INVALID_ARG before anything is launched, and
+ *    bq_last_cuda_error() then names the limit.
+ *  - Memory: the array is a static device variable of libbq.so, so every
+ *    GPU on which the library is used holds those 4 MiB until the process
+ *    exits.  The call itself allocates nothing (no cudaMalloc, no
+ *    cudaFree, no allocating library routine).
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current), once.  Make
+ *    that first call before any stream capture on the device.
+ *  - Sharing: every call on a device uses the same array, and the array
+ *    keeps the last call's contents.  Nothing in it needs to start at zero:
+ *    each call writes every entry it later reads, in stream order.  Calls
+ *    whose work overlaps on the GPU (different streams, or different host
+ *    threads, without ordering between them) race on the array and give
+ *    wrong results; order them, e.g. by using one stream.
+ */
+#define BQ_NOALLOC_MAX_BLOCKS (1 << 20)
+BQ_API bq_status bq_quantize_blockwise_nested_noalloc(const void *x, bq_dtype x_dtype,
+                                  int64_t n, int32_t blocksize, const float *code,
+                                  int32_t code_entries, const float *code2,
+                                  int32_t code2_entries, int32_t blocksize2,
+                                  uint8_t *out, float *absmax2, uint8_t *qabsmax,
+                                  cudaStream_t stream);
+
+/*
  * Inverse of bq_quantize_blockwise_nested, in one launch: block b's scale is
  * rebuilt as A_b = RN(code2[qabsmax[b]] * absmax2[b / blocksize2]) - exactly
  * the fp32 value the statistics' own dequantization gives - and then

@@ -167,3 +167,17 @@ def test_library_has_no_oracle_dependency(L):
     assert "oracle" not in out
     src = open(os.path.join(ROOT, "dequantization_bq_quantize_b200", "__init__.py")).read()
     assert "import oracle" not in src and "from oracle" not in src
+
+
+def test_noalloc_entry_rejects_sizes_beyond_its_array(L):
+    """The allocation-free nested quantize refuses inputs with more blocks
+    than its fixed statistics array before touching the device."""
+    E = bq.BQ_ERR_INVALID_ARG
+    too_many = (bq.BQ_NOALLOC_MAX_BLOCKS + 1) * 64
+    assert bq.bq_quantize_blockwise_nested_noalloc(P, bq.BQ_BF16, too_many, 64, P, 16, P, 256,
+                                                   256, P, P, P, 0) == E
+    assert "BQ_NOALLOC_MAX_BLOCKS" in bq.bq_last_cuda_error()
+    assert bq.bq_quantize_blockwise_nested_noalloc(P, bq.BQ_BF16, 0, 64, P, 16, P, 256, 256, P, P,
+                                                   P, 0) == bq.BQ_OK
+    assert bq.bq_quantize_blockwise_nested_noalloc(P, bq.BQ_BF16, 100, 64, P, 16, P, 16, 256, P, P,
+                                                   P, 0) == E
