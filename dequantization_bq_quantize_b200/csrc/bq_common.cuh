@@ -21,8 +21,22 @@ template <int DT> struct ElemBytes { static constexpr int value = DT == kF32 ? 4
 // bit 1 = a producer gave up waiting for a free stage.
 __device__ uint32_t g_fault;
 
-// A wait on an mbarrier gives up after this many nanoseconds.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// A wait on an mbarrier gives up after this many nanoseconds (2 s; test
+// builds of the fault path set a shorter limit).
+#ifndef BQ_WAIT_LIMIT_NS
+#define BQ_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = BQ_WAIT_LIMIT_NS;
+
+#ifdef BQ_TEST_HOOKS
+// Test builds only (never libbq.so): the producer of the pipelined kernels
+// skips the copy of this tile, so that the consumers' wait for it runs out
+// and the fault path is exercised without any invalid memory access.
+__device__ int64_t g_test_skip_tile = -1;
+__device__ __forceinline__ bool test_skip_tile(int64_t tile) { return tile == g_test_skip_tile; }
+#else
+__device__ __forceinline__ constexpr bool test_skip_tile(int64_t) { return false; }
+#endif
 
 // ---------------------------------------------------------------- widening --
 
@@ -219,9 +233,45 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
+// addresses 16-byte aligned and bytes a multiple of 16.  `pol` is an L2
+// cache policy (createpolicy).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)),
+        "l"(pol)
+      : "memory");
+}
+
+// For data read once (the codes and scales of a dequantization, GGUF
+// blocks): marked evict-first, they leave L2 to the output lines waiting for
+// write-back (n = 2^29 NF4 -> bf16, dequantize alone: about 251 -> 244 us).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // Named barrier over `count` threads (a multiple of 32), id != 0.
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also returns the OR of `v` over the `count` threads.
+__device__ __forceinline__ bool named_sync_or(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void record_fault(uint32_t bit) { atomicOr(&g_fault, bit); }

@@ -59,28 +59,6 @@ struct SSmem {
 template <int E>
 constexpr size_t ssmem_bytes() { return sizeof(SSmem<E>) + 128; }
 
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
-// addresses 16-byte aligned and bytes a multiple of 16.  `pol` is an L2
-// cache policy (createpolicy).
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)),
-        "l"(pol)
-      : "memory");
-}
-
-// The codes and scales are read once: marked evict-first, they leave L2 to
-// the output lines waiting for write-back (n = 2^29 NF4 -> bf16, kernel
-// alone: about 251 -> 244 us).
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-
 template <int QB>
 __device__ __forceinline__ uint2 smem_codes(const uint8_t* base, int chunk) {
   if constexpr (QB == 8) return *reinterpret_cast<const uint2*>(base + 8 * chunk);
@@ -131,6 +109,7 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
             break;
           }
         }
+        if (test_skip_tile(tile)) continue;  // fault-path test builds only
         const uint32_t abytes = (NESTED ? 1u : 4u) * static_cast<uint32_t>(abs_per_tile);
         mbar_arrive_expect_tx(&s.full[st], CODE_BYTES + abytes);
         bulk_load(s.codes[st], p.q + tile * CODE_BYTES, CODE_BYTES, &s.full[st], pol);

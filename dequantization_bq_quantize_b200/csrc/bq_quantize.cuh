@@ -431,12 +431,12 @@ __global__ void __launch_bounds__(kQThreads, 2)
   pdl_release();
   __syncthreads();
 
-  // Under programmatic dependent launch this CTA may start while the previous
-  // kernel on the stream still runs.  The codebook is read and the search
-  // tables are built before waiting for it (the ABI requires the codebook not
-  // to be an output of the immediately preceding library call on the
-  // stream); the input is read and the outputs are written only after the
-  // wait.
+  // Under programmatic dependent launch this CTA may start while earlier
+  // kernels on the stream still run.  The search tables are built from the
+  // codebook before waiting for them, so that the build overlaps their tail;
+  // after the wait the codebook is read again and, if any entry changed (an
+  // earlier kernel wrote it), the tables are built once more.  The input is
+  // read and the outputs are written only after the wait.
   if (warp == 0) {
     pdl_wait();
     if (lane == 0 && p.full_tiles > 0) {
@@ -450,6 +450,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
             break;
           }
         }
+        if (test_skip_tile(tile)) continue;  // fault-path test builds only
         mbar_arrive_expect_tx(&s.full[st], kTileBytes);
         tma_load_2d(s.stage[st], &tmap, 0, static_cast<int32_t>(tile * kTileRows), &s.full[st]);
       }
@@ -463,6 +464,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
   const int ct = threadIdx.x - 32;
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   pdl_wait();
+  // the tables stand only if the codebook, read at L2 after the wait, still
+  // holds the bits they were built from
+  const bool stale = ct < E && __float_as_uint(__ldcg(p.code + ct)) != __float_as_uint(s.tab.c[ct]);
+  if (named_sync_or(1, kQConsumers, stale)) build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   const int mode = s.tab.mode;
   // REMAP: FP4-like 16-entry tables, float select over ranks (bq_search.cuh)
   if (mode == kModeLutF && E == 16 && s.tab.remap8)

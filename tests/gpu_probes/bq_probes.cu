@@ -9,6 +9,8 @@
 //    bisection, built on the device from the caller's table) against a plain
 //    linear scan of the rule |RN(xn - c_j)| minimal, lowest j on ties, for
 //    EVERY float xn in [-1, 1].
+// 3. Ordering: a kernel that writes a buffer late while the next kernel on
+//    the stream has already started under programmatic dependent launch.
 //
 // The plain scan here is written independently of the library's code.
 #include <cstdint>
@@ -198,6 +200,114 @@ __global__ void wait_timeout(int* result) {
   }
 }
 
+// ------------------------------------------------ late writer (PDL) ----
+
+// Launched with programmatic stream serialization: waits for the work before
+// it, lets the next kernel on the stream start launching at once, spins for
+// spin_ns (ended by the timer), then copies count floats from src to dst.  A
+// kernel launched after it the same way runs the part before its own
+// dependent-launch wait while dst still holds the old values.
+// The stores are volatile asm: the timer reads of the spin touch no memory,
+// so plain stores could legally be performed before the spin.
+__global__ void late_writer(float* dst, const float* src, int count, uint64_t spin_ns) {
+  bq::pdl_wait();
+  bq::pdl_release();
+  const uint64_t t0 = bq::globaltimer_ns();
+  while (bq::globaltimer_ns() - t0 < spin_ns) {
+  }
+  for (int i = threadIdx.x; i < count; i += blockDim.x) {
+    const float v = src[i];
+    asm volatile("st.global.f32 [%0], %1;" ::"l"(dst + i), "f"(v) : "memory");
+  }
+}
+
+// Reads p[idx] at L2 before and after its dependent-launch wait.  The first
+// value is put in shared memory behind a barrier before the wait, as the
+// quantize kernel does with the codebook it builds its tables from: a load
+// whose value is only used after the wait may be performed after it.
+__global__ void early_reader(const float* p, int idx, float* out) {
+  __shared__ float before;
+  if (threadIdx.x == 0) before = __ldcg(p + idx);
+  __syncthreads();
+  bq::pdl_wait();
+  if (threadIdx.x == 0) {
+    out[0] = before;
+    out[1] = __ldcg(p + idx);
+  }
+}
+
+// Timestamps (globaltimer, ns) of a late_writer-like kernel and of the kernel
+// launched after it: t[0] writer start, t[1] writer end of spin, t[2] reader
+// start, t[3] reader after its wait.
+__global__ void timed_writer(unsigned long long* t, uint64_t spin_ns) {
+  bq::pdl_wait();
+  bq::pdl_release();
+  const uint64_t t0 = bq::globaltimer_ns();
+  while (bq::globaltimer_ns() - t0 < spin_ns) {
+  }
+  if (threadIdx.x == 0) {
+    t[0] = t0;
+    t[1] = bq::globaltimer_ns();
+  }
+}
+// late_writer and early_reader with timestamps: t[0] writer start, t[1]
+// writer just before its store, t[2] reader start, t[3] reader after its
+// first load reached shared memory, t[4] reader after its wait; t[5], t[6]
+// the bits of the values read before and after the wait.
+__global__ void timed_late_writer(float* dst, const float* src, unsigned long long* t,
+                                  uint64_t spin_ns) {
+  bq::pdl_wait();
+  bq::pdl_release();
+  const uint64_t t0 = bq::globaltimer_ns();
+  while (bq::globaltimer_ns() - t0 < spin_ns) {
+  }
+  const uint64_t t1 = bq::globaltimer_ns();
+  if (threadIdx.x == 0) {
+    const float v = src[1];
+    asm volatile("st.global.f32 [%0], %1;" ::"l"(dst + 1), "f"(v) : "memory");
+    t[0] = t0;
+    t[1] = t1;
+  }
+}
+__global__ void timed_early_reader(const float* p, unsigned long long* t) {
+  __shared__ float before;
+  const uint64_t t2 = bq::globaltimer_ns();
+  if (threadIdx.x == 0) before = __ldcg(p + 1);
+  __syncthreads();
+  const uint64_t t3 = bq::globaltimer_ns();
+  bq::pdl_wait();
+  const uint64_t t4 = bq::globaltimer_ns();
+  if (threadIdx.x == 0) {
+    t[2] = t2;
+    t[3] = t3;
+    t[4] = t4;
+    t[5] = __float_as_uint(before);
+    t[6] = __float_as_uint(__ldcg(p + 1));
+  }
+}
+__global__ void timed_reader(unsigned long long* t) {
+  const uint64_t t2 = bq::globaltimer_ns();
+  bq::pdl_wait();
+  if (threadIdx.x == 0) {
+    t[2] = t2;
+    t[3] = bq::globaltimer_ns();
+  }
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl1(void (*kernel)(KArgs...), cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int g_sms = 0;
 
 cudaError_t reset() {
@@ -287,6 +397,45 @@ __attribute__((visibility("default"))) int probe_search(const float* code, int e
 }
 
 // result[0] = 1 if the wait completed (it must not), result[1] = ms waited.
+// Enqueue late_writer on `stream` (spin at most 0.2 s, at most 4096 floats).
+__attribute__((visibility("default"))) int probe_late_write(float* dst, const float* src,
+                                                            int count,
+                                                            unsigned long long spin_ns,
+                                                            cudaStream_t stream) {
+  if (count < 0 || count > 4096 || spin_ns > 200000000ull) return cudaErrorInvalidValue;
+  return static_cast<int>(launch_pdl1(late_writer, stream, dst, src, count,
+                                      static_cast<uint64_t>(spin_ns)));
+}
+
+// Enqueue early_reader on `stream`: out[0] = p[idx] before its wait, out[1]
+// after (both device pointers).
+__attribute__((visibility("default"))) int probe_early_read(const float* p, int idx, float* out,
+                                                            cudaStream_t stream) {
+  return static_cast<int>(launch_pdl1(early_reader, stream, p, idx, out));
+}
+
+// The two timed kernels back to back on `stream`; t: 4 device words.
+__attribute__((visibility("default"))) int probe_pdl_timing(unsigned long long* t,
+                                                            unsigned long long spin_ns,
+                                                            cudaStream_t stream) {
+  if (spin_ns > 200000000ull) return cudaErrorInvalidValue;
+  cudaError_t e = launch_pdl1(timed_writer, stream, t, static_cast<uint64_t>(spin_ns));
+  if (e == cudaSuccess) e = launch_pdl1(timed_reader, stream, t);
+  return static_cast<int>(e);
+}
+
+// timed_late_writer then timed_early_reader on `stream`; t: 7 device words.
+__attribute__((visibility("default"))) int probe_pdl_timing2(float* dst, const float* src,
+                                                             unsigned long long* t,
+                                                             unsigned long long spin_ns,
+                                                             cudaStream_t stream) {
+  if (spin_ns > 200000000ull) return cudaErrorInvalidValue;
+  cudaError_t e = launch_pdl1(timed_late_writer, stream, dst, src, t,
+                              static_cast<uint64_t>(spin_ns));
+  if (e == cudaSuccess) e = launch_pdl1(timed_early_reader, stream, static_cast<const float*>(dst), t);
+  return static_cast<int>(e);
+}
+
 __attribute__((visibility("default"))) int probe_wait_timeout(int* result) {
   int* d = nullptr;
   cudaError_t e = cudaMalloc(&d, 2 * sizeof(int));
