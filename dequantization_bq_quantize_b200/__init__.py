@@ -219,7 +219,21 @@ def _check(fn, status):
         raise BQError(fn, status, f"{detail} ({extra})" if extra else detail)
 
 
+def _check_fault(fn):
+    """Read and clear the device fault word (this synchronizes the device);
+    raise if a kernel gave up on a bounded wait, which leaves its outputs
+    invalid."""
+    f = bq_device_fault(reset=True)
+    if f:
+        raise BQError(fn, BQ_ERR_CUDA,
+                      f"a kernel gave up waiting (device fault word {f:#x}); outputs are invalid")
+
+
 # --------------------------------------------------------- torch helpers ----
+#
+# Every helper takes check=False.  With check=True it synchronizes after the
+# launch and raises BQError if a kernel gave up on one of its bounded waits
+# (the launch itself succeeded, so nothing else would report it).
 
 def _torch():
     import torch
@@ -250,7 +264,7 @@ def code_bytes(n, entries):
     return (n + 1) // 2 if entries == 16 else n
 
 
-def quantize_blockwise(x, code, blocksize, absmax=None, out=None, stream=None):
+def quantize_blockwise(x, code, blocksize, absmax=None, out=None, stream=None, check=False):
     """Quantize the CUDA tensor x (fp32/fp16/bf16, any shape, flattened).
 
     code: CUDA float32 tensor of 16 or 256 sorted entries.
@@ -268,10 +282,13 @@ def quantize_blockwise(x, code, blocksize, absmax=None, out=None, stream=None):
     _check("bq_quantize_blockwise", bq_quantize_blockwise(
         x.data_ptr(), _dtype_code(x.dtype), n, blocksize, code.data_ptr(), entries,
         absmax.data_ptr(), out.data_ptr(), _stream_handle(stream)))
+    if check:
+        _check_fault("bq_quantize_blockwise")
     return absmax, out
 
 
-def dequantize_blockwise(q, absmax, n, blocksize, code, dtype=None, out=None, stream=None):
+def dequantize_blockwise(q, absmax, n, blocksize, code, dtype=None, out=None, stream=None,
+                         check=False):
     """Inverse of quantize_blockwise: n values of ``dtype`` (default bf16)."""
     torch = _torch()
     _need_cuda(q, "q")
@@ -282,10 +299,12 @@ def dequantize_blockwise(q, absmax, n, blocksize, code, dtype=None, out=None, st
     _check("bq_dequantize_blockwise", bq_dequantize_blockwise(
         q.data_ptr(), absmax.data_ptr(), n, blocksize, code.data_ptr(), code.numel(),
         out.data_ptr(), _dtype_code(out.dtype), _stream_handle(stream)))
+    if check:
+        _check_fault("bq_dequantize_blockwise")
     return out
 
 
-def dequant_gguf(kind, blocks, dtype=None, out=None, stream=None):
+def dequant_gguf(kind, blocks, dtype=None, out=None, stream=None, check=False):
     """GGUF blocks of type ``kind`` (a key of GGUF_TYPES; uint8 CUDA tensor of
     n_blocks * block bytes) -> outputs-per-block * n_blocks values of ``dtype``
     (default bf16)."""
@@ -301,6 +320,8 @@ def dequant_gguf(kind, blocks, dtype=None, out=None, stream=None):
     fn = globals()["bq_dequant_" + kind]
     _check(fn.__name__, fn(blocks.data_ptr(), nblk, out.data_ptr(), _dtype_code(out.dtype),
                            _stream_handle(stream)))
+    if check:
+        _check_fault(fn.__name__)
     return out
 
 
@@ -359,7 +380,7 @@ def dequant_q6_k(blocks, dtype=None, out=None, stream=None):
     return dequant_gguf("q6_k", blocks, dtype, out, stream)
 
 
-def quantize_gguf(kind, x, out=None, stream=None):
+def quantize_gguf(kind, x, out=None, stream=None, check=False):
     """Encode the CUDA tensor x (fp32/fp16/bf16, numel a multiple of 32) as
     GGUF ``kind`` blocks ("q8_0" or "q4_0"): a uint8 tensor of
     numel/32 * block bytes."""
@@ -376,13 +397,15 @@ def quantize_gguf(kind, x, out=None, stream=None):
     fn = globals()["bq_quantize_" + kind]
     _check(fn.__name__, fn(x.data_ptr(), _dtype_code(x.dtype), n, out.data_ptr(),
                            _stream_handle(stream)))
+    if check:
+        _check_fault(fn.__name__)
     return out
 
 
 # -------------------------------------------------- compressed statistics ----
 
 def quantize_blockwise_nested(x, code, blocksize, code2, blocksize2=256, absmax=None, out=None,
-                              absmax2=None, qabsmax=None, stream=None):
+                              absmax2=None, qabsmax=None, stream=None, check=False):
     """Blockwise quantization with compressed statistics: the fp32 absmax array
     of the first pass is itself quantized blockwise with `code2` (the 256-entry
     dynamic 8-bit table) in blocks of `blocksize2`.  Returns (codes, absmax
@@ -406,11 +429,13 @@ def quantize_blockwise_nested(x, code, blocksize, code2, blocksize2=256, absmax=
         x.data_ptr(), _dtype_code(x.dtype), n, blocksize, code.data_ptr(), code.numel(),
         code2.data_ptr(), code2.numel(), blocksize2, absmax.data_ptr(), out.data_ptr(),
         absmax2.data_ptr(), qabsmax.data_ptr(), _stream_handle(stream)))
+    if check:
+        _check_fault("bq_quantize_blockwise_nested")
     return out, qabsmax, absmax2, absmax
 
 
 def dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code, code2, blocksize2=256,
-                                dtype=None, out=None, stream=None):
+                                dtype=None, out=None, stream=None, check=False):
     """Inverse of quantize_blockwise_nested in one launch: each block's scale
     is rebuilt from its code and the second-level scale inside the kernel."""
     torch = _torch()
@@ -423,6 +448,8 @@ def dequantize_blockwise_nested(q, qabsmax, absmax2, n, blocksize, code, code2, 
         q.data_ptr(), qabsmax.data_ptr(), absmax2.data_ptr(), n, blocksize, code.data_ptr(),
         code.numel(), code2.data_ptr(), code2.numel(), blocksize2, out.data_ptr(),
         _dtype_code(out.dtype), _stream_handle(stream)))
+    if check:
+        _check_fault("bq_dequantize_blockwise_nested")
     return out
 
 
@@ -432,7 +459,7 @@ _side_streams = {}
 
 
 def quantize_blockwise_host(x_host, code, blocksize, code2=None, blocksize2=256,
-                            chunk_elements=1 << 24, staging=None, device=None):
+                            chunk_elements=1 << 24, staging=None, device=None, check=False):
     """Quantize a CPU tensor (pin it for overlap) straight into device outputs,
     copying and quantizing chunk by chunk over two streams: torch's current
     stream and a side stream, joined back into the current stream.  Returns
@@ -460,13 +487,14 @@ def quantize_blockwise_host(x_host, code, blocksize, code2=None, blocksize2=256,
     side = _side_streams.get(dev.index)
     if side is None:
         side = _side_streams[dev.index] = torch.cuda.Stream(device=dev)
-    side.wait_stream(cur)  # outputs and staging were made on the current stream
     _check("bq_quantize_blockwise_host", bq_quantize_blockwise_host(
         x_host.data_ptr(), _dtype_code(x_host.dtype), n, blocksize, code.data_ptr(), code.numel(),
         code2.data_ptr() if code2 is not None else None, 256, blocksize2, absmax.data_ptr(),
         out.data_ptr(), absmax2.data_ptr() if absmax2 is not None else None,
         qabsmax.data_ptr() if qabsmax is not None else None, staging.data_ptr(),
         staging.numel(), chunk_elements, cur.cuda_stream, side.cuda_stream))
+    if check:
+        _check_fault("bq_quantize_blockwise_host")
     if code2 is None:
         return absmax, out
     return out, qabsmax, absmax2, absmax

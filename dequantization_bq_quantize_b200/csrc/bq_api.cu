@@ -590,6 +590,14 @@ bq_status bq_quantize_blockwise_host(const void* x_host, bq_dtype x_dtype, int64
   if (two) {
     cudaError_t e = cudaEventCreateWithFlags(&joined, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e, "pipeline event");
+    // stream1's chunks start only after the work already queued on stream0
+    // (which may still use the outputs or the staging buffer)
+    e = cudaEventRecord(joined, stream0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream1, joined, 0);
+    if (e != cudaSuccess) {
+      cudaEventDestroy(joined);
+      return cuda_fail(e, "pipeline entry ordering");
+    }
   }
   bq_status st = BQ_OK;
   for (int64_t i = 0; i < chunks && st == BQ_OK; ++i) {
@@ -615,7 +623,8 @@ bq_status bq_quantize_blockwise_host(const void* x_host, bq_dtype x_dtype, int64
                                         absmax + b0, o, s);
   }
   if (two) {
-    // stream0 continues only after stream1's chunks
+    // stream0 continues only after stream1's chunks (the event is re-recorded:
+    // cudaStreamWaitEvent above captured its first recording already)
     cudaError_t e = cudaEventRecord(joined, stream1);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(stream0, joined, 0);
     if (e != cudaSuccess && st == BQ_OK) st = cuda_fail(e, "pipeline join");
@@ -735,5 +744,14 @@ bq_status bq_device_fault(uint32_t* fault, int32_t reset) {
 }
 
 int32_t bq_abi_version(void) { return BQ_ABI_VERSION; }
+
+#ifdef BQ_TEST_HOOKS
+// Test builds only (not declared in bq.h, not in libbq.so): choose the tile
+// whose copy the pipelined kernels' producers skip (-1: none).
+__attribute__((visibility("default"))) bq_status bq_test_skip_tile(int64_t tile) {
+  const cudaError_t e = cudaMemcpyToSymbol(bq::g_test_skip_tile, &tile, sizeof(tile));
+  return e == cudaSuccess ? BQ_OK : cuda_fail(e, "setting the test hook");
+}
+#endif
 
 }  // extern "C"

@@ -84,12 +84,11 @@ typedef enum bq_dtype {
  *                high nibble of byte i, element 2i+1 in the low nibble (0 if it
  *                does not exist); 256 entries: n bytes, one code per element.
  * Inputs must be finite (non-finite values are outside the contract).
- * Ordering: the kernel starts under programmatic dependent launch and reads
- * `code` (to build its search tables) before waiting for the kernel launched
- * just before it on `stream`; everything else is read and written after that
- * wait.  So `code` must not be an output of the immediately preceding
- * library call on the same stream (copies, and kernels of other libraries,
- * are always complete before it is read).
+ * Ordering: everything the call reads, `code` included, may be written by
+ * any earlier work on `stream`, library calls included.  (The kernel starts
+ * under programmatic dependent launch and builds its search tables from
+ * `code` while earlier kernels finish; after waiting for them it reads
+ * `code` again and rebuilds the tables if any entry changed.)
  */
 BQ_API bq_status bq_quantize_blockwise(const void *x, bq_dtype x_dtype, int64_t n,
                                 int32_t blocksize, const float *code,
@@ -200,8 +199,10 @@ BQ_API bq_status bq_dequantize_blockwise_nested(const uint8_t *q, const uint8_t 
  * after its copy on the same stream (with compressed statistics when code2 is
  * not NULL), so one chunk's copy overlaps the other's quantization.  The
  * outputs are bit-identical to one bq_quantize_blockwise(_nested) call on the
- * whole input.  At return, stream0 has been made to wait for stream1's work:
- * the outputs are complete in stream0's order.
+ * whole input.  Ordering: stream1's first copy waits for the work queued on
+ * stream0 before the call, and at return stream0 has been made to wait for
+ * stream1's work, so the whole call behaves as work on stream0: the outputs
+ * are complete in stream0's order.
  * Exception to the common contract: this call reads host memory and creates
  * (and releases) one CUDA event per call.
  *   x_host        host, n elements of x_dtype.  Pinned (page-locked) memory
