@@ -5,7 +5,6 @@ must match exactly (the contract allows 1 ulp for bf16/fp16; the kernels do the
 same single product and rounding, so exact equality is asserted).
 """
 import ctypes
-import time
 
 import numpy as np
 import pytest
@@ -15,7 +14,7 @@ import dequantization_bq_quantize_b200 as bq
 import oracle
 from bq_inputs import codebooks, synth
 
-from gpu_util import Guarded, device_copy, np_bits, sample_blocks
+from gpu_util import Guarded, device_copy, np_bits
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -191,44 +190,6 @@ def test_zero_length_and_bad_arguments():
     assert bq.bq_dequant_q8_0(0, 5, out.data_ptr(), bq.BQ_BF16, 0) == bq.BQ_ERR_INVALID_ARG
 
 
-# ---------------------------------------------------------- stream order --
-
-def _ordering_case(use_callers_stream):
-    """A producer fills the input on a non-blocking stream held back by a
-    ~25 ms device-side delay, then quantize is called at once."""
-    n, bs = 1 << 20, 64
-    code = code_dev(TABLES["nf4"])
-    x_final = small_input(n, "bf16", bs, seed=5)
-    src = torch.from_numpy(x_final.view(np.int16)).cuda()
-    x = torch.zeros(n, dtype=torch.int16, device="cuda")
-    amax = torch.empty((n + bs - 1) // bs, device="cuda")
-    out = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
-    torch.cuda.synchronize()
-    s = torch.cuda.Stream()  # non-blocking with respect to the legacy stream
-    with torch.cuda.stream(s):
-        torch.cuda._sleep(50_000_000)  # bounded spin, tens of ms
-        x.copy_(src)
-        st = bq.bq_quantize_blockwise(x.data_ptr(), bq.BQ_BF16, n, bs, code.data_ptr(), 16,
-                                      amax.data_ptr(), out.data_ptr(),
-                                      s.cuda_stream if use_callers_stream else 0)
-    assert st == bq.BQ_OK
-    torch.cuda.synchronize()
-    oa, oo = oracle.quantize_blockwise(x_final, "bf16", bs, TABLES["nf4"])
-    return np.array_equal(amax.cpu().numpy(), oa) and np.array_equal(out.cpu().numpy(), oo)
-
-
-def test_respects_callers_stream():
-    """Ordering regression of the stream-aware entry points (bitsandbytes
-    PR #2052): on the caller's stream the quantizer sees the final input."""
-    assert _ordering_case(True)
-
-
-def test_ordering_case_detects_wrong_stream():
-    """Control: the same sequence with the legacy stream reads stale input,
-    so the case above can tell the two apart."""
-    assert not _ordering_case(False)
-
-
 # ------------------------------------------------------------------ GGUF --
 
 @pytest.mark.parametrize("kind", list(bq.GGUF_TYPES))
@@ -376,10 +337,27 @@ def test_gguf_encode_rejects_bad_arguments():
 
 # ------------------------------------------------------ full-size configs --
 
-def _run_full(x_cpu, dtype, bs, name, sample=3000, seed=0):
-    """Full-size run through the torch helpers (same launch configuration as
-    the benchmark), checked on sampled whole blocks against the oracle and on
-    all blocks for properties that hold at any size."""
+THREADS = oracle.host_threads()
+
+
+def _bits(a):
+    """Raw bit patterns, so that -0 / +0 and NaN payloads count as different."""
+    a = np.ascontiguousarray(a)
+    return a.view({4: np.uint32, 2: np.uint16, 1: np.uint8}[a.itemsize])
+
+
+def _assert_same(what, got, want):
+    g, w = _bits(got), _bits(want)
+    assert g.shape == w.shape, (what, g.shape, w.shape)
+    bad = np.flatnonzero(g != w)
+    assert bad.size == 0, f"{what}: {bad.size} of {g.size} differ, first at {bad[:5]}"
+
+
+def _run_full(x_cpu, dtype, bs, name):
+    """Full-size run through the torch helpers (the launch configuration the
+    benchmark times), then EVERY absmax, code byte and dequantized value
+    against the oracle (driven over disjoint block ranges on all host
+    threads; blocks are independent, so that is the single call's result)."""
     table = TABLES[name]
     code = code_dev(table)
     n = x_cpu.numel()
@@ -387,24 +365,14 @@ def _run_full(x_cpu, dtype, bs, name, sample=3000, seed=0):
     amax, q = bq.quantize_blockwise(x, code, bs)
     y = bq.dequantize_blockwise(q, amax, n, bs, code, dtype=x.dtype)
     torch.cuda.synchronize()
-    nb = amax.numel()
-    # properties at any size: absmax is max|x| of each block, dequant of the
-    # block's extreme element is +-absmax * (table end) ...
-    xf = x.float()
-    full_blocks = n // bs
-    ref_amax = xf[: full_blocks * bs].abs().view(full_blocks, bs).amax(dim=1)
-    assert torch.equal(amax[:full_blocks], ref_amax)
-    # sampled blocks against the oracle
-    xh = np_bits(x_cpu)
     ah, qh, yh = amax.cpu().numpy(), q.cpu().numpy(), np_bits(y.cpu())
-    for b in sample_blocks(nb, sample, seed):
-        lo, hi = b * bs, min(n, (b + 1) * bs)
-        oa, oo = oracle.quantize_blockwise(xh[lo:hi], dtype, bs, table)
-        assert ah[b] == oa[0]
-        q0 = lo // 2 if table.size == 16 else lo
-        assert np.array_equal(qh[q0:q0 + oo.size], oo), b
-        oy = oracle.dequantize_blockwise(oo, oa, hi - lo, bs, table, dtype)
-        assert np.array_equal(yh[lo:hi], oy), b
+    del x, amax, q, y
+    xh = np_bits(x_cpu)
+    oa, oq = oracle.quantize_blockwise_threaded(xh, dtype, bs, table, THREADS)
+    _assert_same("absmax", ah, oa)
+    _assert_same("codes", qh, oq)
+    oy = oracle.dequantize_blockwise_threaded(oq, oa, n, bs, table, dtype, THREADS)
+    _assert_same("dequantized", yh, oy)
 
 
 def test_config_small_fp32_nf4_full():
@@ -416,27 +384,37 @@ def test_config_small_fp32_nf4_full():
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 @pytest.mark.parametrize("name", ["nf4", "fp4", "dyn8"])
-def test_config_sweep_sampled(dtype, name):
-    """The 45-cell sweep at n = 8388608 + 37 with one all-zero block."""
+def test_config_sweep_full(dtype, name):
+    """The 45-cell sweep at n = 8388608 + 37 with one all-zero block: every
+    output of every cell (dequantized to the cell's input dtype)."""
     for i, bs in enumerate((32, 64, 256, 1024, 4096)):
         cell = ["f16", "bf16", "f32"].index(dtype) * 15 + ["nf4", "fp4", "dyn8"].index(name) * 5 + i
         x = synth.sweep(dtype, bs, seed=1 + cell)
-        _run_full(x, dtype, bs, name, sample=400, seed=cell)
+        _run_full(x, dtype, bs, name)
 
 
-def test_config_large_bf16_nf4():
-    """bf16 n = 2^29 (1 GiB) N(0, 0.02) with 0.1% outliers, NF4, blocksize 64."""
+def test_config_large_bf16_nf4_full():
+    """bf16 n = 2^29 (1 GiB) N(0, 0.02) with 0.1% outliers, NF4, blocksize 64:
+    every output (the persistent rings wrap hundreds of times per CTA)."""
     x, count = synth.large_outliers()
     assert 0.0009 < count / x.numel() < 0.0011
-    _run_full(x, "bf16", 64, "nf4", sample=4000, seed=3)
+    _run_full(x, "bf16", 64, "nf4")
 
 
-def test_config_llama_weight_set_sampled():
-    """A few of the Llama-3-8B-shaped matrices (bf16 N(0, 0.02), NF4 bs 64)."""
+def test_config_llama_weight_set_full():
+    """All 224 Llama-3-8B-shaped matrices (bf16 N(0, 0.02), NF4 blocksize 64),
+    every output of each; the next matrix's input is drawn while the current
+    one is checked."""
+    from concurrent.futures import ThreadPoolExecutor
     mats = synth.llama_matrices(layers=32)
-    for layer, i, name, r, c, seed in (mats[0], mats[4], mats[6], mats[-1]):
-        x = synth.normal(r * c, "bf16", seed, std=0.02)
-        _run_full(x, "bf16", 64, "nf4", sample=300, seed=seed)
+    draw = lambda m: synth.normal(m[3] * m[4], "bf16", m[5], std=0.02)  # noqa: E731
+    with ThreadPoolExecutor(1) as ex:
+        nxt = ex.submit(draw, mats[0])
+        for k, m in enumerate(mats):
+            x = nxt.result()
+            if k + 1 < len(mats):
+                nxt = ex.submit(draw, mats[k + 1])
+            _run_full(x, "bf16", 64, "nf4")
 
 
 # ---------------------------------------------------------- exhaustive ----
@@ -629,29 +607,71 @@ def test_nested_rejects_bad_arguments():
 
 # ------------------------------------------------------ host-input pipeline --
 
+def _oracle_host(xh, dtype, bs, bs2, nested):
+    oa, oq = oracle.quantize_blockwise(xh, dtype, bs, TABLES["nf4"])
+    if not nested:
+        return oa, oq
+    oa2, oqa = oracle.quantize_blockwise(oa, "f32", bs2, TABLES["dyn8"])
+    return oq, oqa, oa2, oa
+
+
 @pytest.mark.parametrize("nested", [False, True])
 @pytest.mark.parametrize("pinned", [True, False])
-def test_host_pipeline_matches_device_call(nested, pinned):
-    """The two-stream host pipeline gives the bytes of one call on the whole
-    device-resident input: several chunks and a ragged tail, both halves of
-    the staging buffer reused more than once."""
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_host_pipeline_against_oracle(nested, pinned, dtype):
+    """The two-stream host pipeline against the oracle (and against one call
+    on the whole device-resident input): several chunks and a ragged last
+    chunk, both halves of the staging buffer reused more than once, so every
+    chunk's offsets into absmax, the codes and the second-level statistics
+    are checked."""
     bs, bs2 = 64, 256
     chunk = bs * bs2 * 3                        # 49152 elements
     n = chunk * 5 + 1000 * bs + 17              # 5 whole chunks and a partial one
-    x = synth.with_zero_block(synth.normal(n, "bf16", seed=5 + nested), bs)
+    x = synth.with_zero_block(synth.normal(n, dtype, seed=5 + nested), bs)
     xh = x.pin_memory() if pinned else x
     nf4, dyn = code_dev(TABLES["nf4"]), code_dev(TABLES["dyn8"])
     if nested:
         got = bq.quantize_blockwise_host(xh, nf4, bs, dyn, bs2, chunk_elements=chunk)
-        want = bq.quantize_blockwise_nested(x.cuda(), nf4, bs, dyn, bs2)
+        dev_call = bq.quantize_blockwise_nested(x.cuda(), nf4, bs, dyn, bs2)
     else:
         got = bq.quantize_blockwise_host(xh, nf4, bs, chunk_elements=chunk)
-        want = bq.quantize_blockwise(x.cuda(), nf4, bs)
+        dev_call = bq.quantize_blockwise(x.cuda(), nf4, bs)
     torch.cuda.synchronize()
-    assert len(got) == len(want)
-    for g, w in zip(got, want):
-        assert torch.equal(g, w)
+    want = _oracle_host(np_bits(x), dtype, bs, bs2, nested)
+    assert len(got) == len(want) == len(dev_call)
+    for i, (g, w, d) in enumerate(zip(got, want, dev_call)):
+        _assert_same(f"output {i}", g.cpu().numpy(), w)
+        assert torch.equal(g, d)
     assert bq.bq_device_fault() == 0
+
+
+def test_host_pipeline_waits_for_work_queued_on_stream0():
+    """Work queued on stream0 before the call - here a delayed fill of the
+    output buffers - lands before the second stream's chunks write them: the
+    C call orders its second stream after stream0 by itself (the second
+    stream is never synchronised with stream0 by the caller)."""
+    bs = 64
+    chunk = 1 << 16
+    n = 7 * chunk + 333
+    x = synth.normal(n, "bf16", seed=17).pin_memory()
+    nf4 = code_dev(TABLES["nf4"])
+    want_a, want_q = _oracle_host(np_bits(x), "bf16", bs, 256, False)
+    a = torch.empty(want_a.size, device="cuda")
+    q = torch.empty(want_q.size, dtype=torch.uint8, device="cuda")
+    staging = torch.empty(2 * chunk * 2, dtype=torch.uint8, device="cuda")
+    s0, s1 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s0):
+        torch.cuda._sleep(50_000_000)        # a bounded spin, tens of ms
+        a.fill_(-1.0)
+        q.fill_(0xFF)
+    assert bq.bq_quantize_blockwise_host(x.data_ptr(), bq.BQ_BF16, n, bs, nf4.data_ptr(), 16,
+                                         None, 0, 0, a.data_ptr(), q.data_ptr(), None, None,
+                                         staging.data_ptr(), staging.numel(), chunk,
+                                         s0.cuda_stream, s1.cuda_stream) == bq.BQ_OK
+    torch.cuda.synchronize()
+    _assert_same("absmax", a.cpu().numpy(), want_a)
+    _assert_same("codes", q.cpu().numpy(), want_q)
 
 
 def test_host_pipeline_single_stream_and_one_chunk():
@@ -690,3 +710,20 @@ def test_host_pipeline_single_stream_and_one_chunk():
                                          staging.data_ptr(), staging.numel(), 65536 + 128, s,
                                          s) == E
     assert bq.bq_device_fault() == 0
+
+
+def test_torch_helpers_check_option():
+    """check=True synchronizes and reads the fault word after the launch; a
+    clean run returns the same outputs as without it."""
+    x = synth.normal(3 * 8192 + 101, "bf16", seed=23).cuda()
+    nf4, dyn = code_dev(TABLES["nf4"]), code_dev(TABLES["dyn8"])
+    a, q = bq.quantize_blockwise(x, nf4, 64, check=True)
+    a0, q0 = bq.quantize_blockwise(x, nf4, 64)
+    assert torch.equal(a, a0) and torch.equal(q, q0)
+    y = bq.dequantize_blockwise(q, a, x.numel(), 64, nf4, check=True)
+    assert torch.equal(y, bq.dequantize_blockwise(q, a, x.numel(), 64, nf4))
+    qn, qa, a2, _ = bq.quantize_blockwise_nested(x, nf4, 64, dyn, 256, check=True)
+    bq.dequantize_blockwise_nested(qn, qa, a2, x.numel(), 64, nf4, dyn, 256, check=True)
+    blocks = bq.quantize_gguf("q4_0", x[: x.numel() // 32 * 32], check=True)
+    bq.dequant_gguf("q4_0", blocks, check=True)
+    bq.quantize_blockwise_host(x.cpu(), nf4, 64, chunk_elements=8192, check=True)
