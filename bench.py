@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--n", type=int, default=N_LARGE, help="elements of the quantize input")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sweep / weight-set / other-codebook figures of the default line")
     ap.add_argument("--only", choices=["all", "quantize", "dequantize", "q8_0", "q4_0"],
                     default="all", help="run one kernel per step (profiling aid)")
     ap.add_argument("--codebook", choices=["nf4", "fp4", "dyn8"], default="nf4",
@@ -306,6 +308,242 @@ def _pct(sorted_ts, f):
     return sorted_ts[min(len(sorted_ts) - 1, int(f * (len(sorted_ts) - 1) + 0.5))]
 
 
+# ------------------------------------------------------------- checking --
+
+def _raw_bits(a):
+    """Bit patterns of a numpy array (so -0 / +0 count as different)."""
+    a = np.ascontiguousarray(a)
+    return a.view({4: np.uint32, 2: np.uint16, 1: np.uint8}[a.itemsize])
+
+
+def _host_bits(t):
+    t = t.cpu()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        t = t.view(torch.int16)
+    return _raw_bits(t.numpy())
+
+
+def verify_step(w, names, world):
+    """Every output of the last timed step against the oracle: absmax, codes
+    and the dequantized tensor of the 2^29-element input, and both GGUF
+    matrices, bit for bit.  The oracle runs over disjoint block ranges on the
+    host threads (blocks are independent, so this is the single call's
+    result).  Returns (summary, the oracle's outputs) - (None, None) for the
+    one-kernel profiling runs - and raises if any output differs."""
+    if names != ["quantize", "dequantize", "q8_0", "q4_0"]:
+        return None, None
+    import oracle
+    threads = max(1, oracle.host_threads() // world)
+    t0 = time.perf_counter()
+    table = codebooks.get(w.codebook)
+    oa, oq = oracle.quantize_blockwise_threaded(synth.to_numpy_bits(w.x_cpu), "bf16", BS, table,
+                                                threads)
+    expected = {
+        "absmax": oa, "codes": oq,
+        "dequantize": oracle.dequantize_blockwise_threaded(oq, oa, w.n, BS, table, "bf16",
+                                                           threads),
+        "q8_0": oracle.dequant_gguf("q8_0", w.q8_cpu.numpy(), "bf16"),
+        "q4_0": oracle.dequant_gguf("q4_0", w.q4_cpu.numpy(), "bf16"),
+    }
+    got = {"absmax": w.absmax, "codes": w.q, "dequantize": w.y, "q8_0": w.y8, "q4_0": w.y4}
+    differ, values = {}, 0
+    for k, t in got.items():
+        g, e = _host_bits(t), _raw_bits(expected[k])
+        differ[k] = int(np.count_nonzero(g != e)) if g.shape == e.shape else int(g.size)
+        values += g.size
+    worst = max_over_ranks(float(sum(differ.values())), world)
+    if worst != 0:
+        raise RuntimeError(f"bench: outputs of the timed step differ from the oracle: {differ}")
+    return {"ok": True, "against": "oracle", "outputs": list(got), "values_compared": values,
+            "values_differing": 0, "threads": threads,
+            "seconds": round(time.perf_counter() - t0, 2),
+            "what": "every output of the last timed step, bit for bit"}, expected
+
+
+# ---------------------------------------------- figures beyond the step --
+
+def _event_ms(fn, reps=5):
+    """Median device time (ms) of fn() over `reps` calls, each bracketed by
+    its own CUDA events on the current stream.  For calls of hundreds of
+    microseconds or more: event timestamps here advance in steps of about
+    2 us."""
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ts)
+    return ms[len(ms) // 2]
+
+
+def _flush_graph_ms(flush, reps):
+    """Replay time (ms) of a CUDA graph of `reps` reads of the flush buffer."""
+    g = _capture(lambda: [flush.sum() for _ in range(reps)])
+    ms = _replay_ms(g)
+    del g
+    return ms
+
+
+def _flushed_ms(fn, flush, reps, base_ms):
+    """Device time (ms) of one fn() call that starts with a cold, clean L2:
+    `reps` pairs (read the flush buffer, fn()) captured in one CUDA graph,
+    minus `base_ms` (the same number of flush reads alone), divided by reps.
+    Reading (not writing) the buffer evicts the inputs and leaves L2 clean, so
+    the call pays no write-back of the flush; the graph removes host launch
+    gaps, and dividing by reps the event resolution."""
+    def both():
+        for _ in range(reps):
+            flush.sum()
+            fn()
+    g = _capture(both)
+    ms = _replay_ms(g)
+    del g
+    return max((ms - base_ms) / reps, 0.0)
+
+
+def _codebook_figures(w, peak):
+    """FP4 and dyn8 (256-entry) quantize + dequantize of the step's 1 GiB bf16
+    input, blocksize 64 (the input is larger than L2: no flush)."""
+    bq = w.bq
+    dev = w.x.device
+    rows = {}
+    q8 = torch.empty(w.n, dtype=torch.uint8, device=dev)
+    for name in ("fp4", "dyn8"):
+        code = torch.from_numpy(codebooks.get(name)).to(dev)
+        q = w.q if code.numel() == 16 else q8
+        nbytes = quant_bytes(w.n, BS, entries=code.numel())
+        tq = _event_ms(lambda: bq.quantize_blockwise(w.x, code, BS, absmax=w.absmax, out=q))
+        td = _event_ms(lambda: bq.dequantize_blockwise(q, w.absmax, w.n, BS, code, out=w.y))
+        rows[name] = {"quantize_us": round(tq * 1e3, 1),
+                      "quantize_frac": round(nbytes / (tq / 1e3) / 1e9 / peak, 4),
+                      "dequantize_us": round(td * 1e3, 1),
+                      "dequantize_frac": round(nbytes / (td / 1e3) / 1e9 / peak, 4),
+                      "bytes": nbytes}
+    del q8
+    return rows
+
+
+def sweep_cells(peak, reps=10):
+    """The 45-cell sweep: {fp16, bf16, fp32} x {NF4, FP4, dyn8} x blocksize
+    {32, 64, 256, 1024, 4096} at n = 8388608 + 37, N(0, 1) with one all-zero
+    block (block nb // 2), drawn on the device from a generator seeded with
+    1 + cell.  Quantize, and dequantize to the input dtype, each timed on its
+    own after an L2 flush (the cell's tensors fit in L2; _flushed_ms)."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.zeros(80 << 20, dtype=torch.int32, device=dev)   # 320 MiB
+    base = _flush_graph_ms(flush, reps)
+    n = synth.SWEEP_N
+    cells = []
+    ci = 0
+    for dtype in ("f16", "bf16", "f32"):
+        for name in ("nf4", "fp4", "dyn8"):
+            code = torch.from_numpy(codebooks.get(name)).to(dev)
+            for bs in (32, 64, 256, 1024, 4096):
+                g = torch.Generator(device=dev)
+                g.manual_seed(1 + ci)
+                x = torch.randn(n, generator=g, device=dev).to(synth.TORCH_DTYPES[dtype])
+                nb = (n + bs - 1) // bs
+                x[(nb // 2) * bs: min(n, (nb // 2 + 1) * bs)] = 0
+                a, q = bq.quantize_blockwise(x, code, bs)
+                y = torch.empty_like(x)
+                nbytes = quant_bytes(n, bs, x.element_size(), code.numel())
+                tq = _flushed_ms(lambda: bq.quantize_blockwise(x, code, bs, absmax=a, out=q),
+                                 flush, reps, base)
+                td = _flushed_ms(lambda: bq.dequantize_blockwise(q, a, n, bs, code, out=y),
+                                 flush, reps, base)
+                cells.append({"dtype": dtype, "codebook": name, "blocksize": bs,
+                              "quantize_us": round(tq * 1e3, 1),
+                              "quantize_gbs": round(nbytes / (tq / 1e3) / 1e9, 1),
+                              "dequantize_us": round(td * 1e3, 1),
+                              "dequantize_gbs": round(nbytes / (td / 1e3) / 1e9, 1)})
+                ci += 1
+    del flush
+    fr = lambda k: sorted(c[k] / peak for c in cells)  # noqa: E731
+    summary = {k: {"min": round(fr(k)[0], 4), "median": round(fr(k)[len(cells) // 2], 4),
+                   "max": round(fr(k)[-1], 4)} for k in ("quantize_gbs", "dequantize_gbs")}
+    return cells, summary
+
+
+def llama_weight_set(steps=3, warmup=1):
+    """The 224 weight matrices of a Llama-3-8B-shaped model (32 layers), bf16
+    N(0, 0.02) drawn on the device from a generator seeded per matrix; NF4
+    blocksize 64 quantize then dequantize of every matrix back to back on one
+    stream, eager and as one CUDA-graph replay (the 448 launches captured
+    once).  Returns the figures and the total bytes."""
+    import dequantization_bq_quantize_b200 as bq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    code = torch.from_numpy(codebooks.nf4()).to(dev)
+    mats, outs = [], []
+    total = 0
+    for layer, i, name, r, c, seed in synth.llama_matrices():
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        x = torch.randn(r * c, generator=g, device=dev, dtype=torch.float32).mul_(0.02).to(
+            torch.bfloat16)
+        n = x.numel()
+        a = torch.empty((n + BS - 1) // BS, dtype=torch.float32, device=dev)
+        q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        y = torch.empty_like(x)
+        mats.append(x)
+        outs.append((a, q, y))
+        total += 2 * quant_bytes(n, BS)
+
+    def everything():
+        for x, (a, q, y) in zip(mats, outs):
+            bq.quantize_blockwise(x, code, BS, absmax=a, out=q)
+            bq.dequantize_blockwise(q, a, x.numel(), BS, code, out=y)
+
+    for _ in range(max(1, warmup)):
+        everything()
+    torch.cuda.synchronize()
+    ms_eager = _event_ms(everything, max(1, steps))
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            everything()
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    ms = _event_ms(graph.replay, max(1, steps))
+    del graph
+    return {"matrices": len(mats), "elements": sum(m.numel() for m in mats), "bytes": total,
+            "eager_ms": round(ms_eager, 3), "graph_ms": round(ms, 3),
+            "graph_gbs": round(total / (ms / 1e3) / 1e9, 1),
+            "eager_gbs": round(total / (ms_eager / 1e3) / 1e9, 1)}
+
+
+def run_extras(w):
+    """Figures beyond the step, reported next to `value` (not part of it):
+    the 45-cell sweep, the Llama-3-8B-shaped weight set and the 1 GiB
+    quantize / dequantize with the FP4 and dyn8 tables, each against the
+    measured copy bandwidth.  The fault word is checked after them."""
+    peak, kind = measured_peaks()
+    t0 = time.perf_counter()
+    other = _codebook_figures(w, peak)
+    cells, summary = sweep_cells(peak)
+    llama = llama_weight_set()
+    llama["graph_frac"] = round(llama["graph_gbs"] / peak, 4)
+    llama["eager_frac"] = round(llama["eager_gbs"] / peak, 4)
+    fault = w.bq.bq_device_fault(reset=True)
+    if fault:
+        raise SystemExit(f"bench: the fault word was set during the extra figures ({fault:#x})")
+    torch.cuda.empty_cache()
+    return {"codebooks_1gib": other,
+            "sweep": {"n": synth.SWEEP_N, "l2": "flushed (320 MiB read) before every call",
+                      "frac_summary": summary, "cells": cells},
+            "llama_weight_set": llama,
+            "extras_peak": f"{peak} GB/s {kind}",
+            "extras_seconds": round(time.perf_counter() - t0, 1)}
+
+
 # -------------------------------------------------------------------- ours --
 
 class Workload:
@@ -391,6 +629,13 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier(world)
+    # a kernel that gave up on a bounded wait returns early and would make the
+    # step look faster: such a run gives no result
+    fault = w.bq.bq_device_fault(reset=True)
+    if max_over_ranks(float(fault), world) != 0:
+        raise SystemExit(f"bench: the fault word was set during the timed region ({fault:#x}) "
+                         "- a kernel gave up waiting; no result is reported")
+    verification, expected = verify_step(w, names, world)
     total_ms = ev[0][0].elapsed_time(ev[-1][-1])
     per_kernel = {k: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)]
                   for i, k in enumerate(names)}
@@ -401,7 +646,11 @@ def run_ours(args, rank, world, local):
     # ---- end to end: host buffers in, results back to the host, every step
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, names, stream, sh, byts, world)
+        e2e = run_e2e(args, w, names, stream, sh, byts, world, expected)
+
+    extras = None
+    if world == 1 and not args.no_extras and args.only == "all" and args.codebook == "nf4":
+        extras = run_extras(w)
 
     peak, peak_kind = measured_peaks()
     kern = {}
@@ -443,13 +692,17 @@ def run_ours(args, rank, world, local):
             "pct_of_nominal_8tbs": {k: round(v["gbs"] / 8000.0, 4) for k, v in kern.items()},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "verified": verification is not None and verification["ok"],
+            "verification": verification,
             "gpu_launches": len(names) * args.steps,
             "clocks": clocks,
         }
+        if extras:
+            line.update(extras)
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, w, names, stream, sh, byts, world, chunks=8):
+def run_e2e(args, w, names, stream, sh, byts, world, expected, chunks=8):
     """Same step through the public API with host buffers, every step: pinned
     host->device copy of the step's inputs and device->host copy of all its
     results inside the timed region.  The work is cut into `chunks` pieces on
@@ -557,15 +810,22 @@ def run_e2e(args, w, names, stream, sh, byts, world, chunks=8):
     e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
-    # the pipelined, chunked calls must give the device-resident results
-    for host, dev in ((ah, w.absmax), (qh, w.q), (yh, w.y), (y8h, w.y8), (y4h, w.y4)):
-        k = min(dev.numel(), 1 << 20)
-        if not (torch.equal(host[:k], dev[:k].cpu()) and torch.equal(host[-k:], dev[-k:].cpu())):
-            raise RuntimeError("end-to-end results differ from the device-resident run")
+    # every output the pipelined, chunked calls brought back to the host must
+    # equal the oracle's (whole arrays)
+    checked = 0
+    if expected is not None:
+        for key, host in (("absmax", ah), ("codes", qh), ("dequantize", yh), ("q8_0", y8h),
+                          ("q4_0", y4h)):
+            if key not in expected:
+                continue
+            if not np.array_equal(_host_bits(host), _raw_bits(expected[key])):
+                raise RuntimeError(f"end-to-end {key} differs from the oracle")
+            checked += host.numel()
     total = sum(byts.values()) * world
     return {"value": round(total / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
-            "steps": steps, "pipeline": f"{len(ranges)} chunks over 3 streams (in / kernels / out)"}
+            "steps": steps, "pipeline": f"{len(ranges)} chunks over 3 streams (in / kernels / out)",
+            "outputs_checked_against_oracle": checked}
 
 
 # ------------------------------------------------------ informational ---
@@ -652,86 +912,17 @@ def _graph_timed(fn, reps=50):
 
 
 def run_sweep(args):
-    """45 cells: {fp16, bf16, fp32} x {NF4, FP4, dyn8} x bs {32, 64, 256, 1024,
-    4096} at n = 8388608 + 37 with one all-zero block; quantize and dequantize
-    (to the input dtype) timed separately with a 320 MiB L2 flush before each
-    repetition (the tensors fit in L2)."""
-    import dequantization_bq_quantize_b200 as bq
-    dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(320 << 20, dtype=torch.uint8, device=dev)
-    cells = []
-    ci = 0
-    for dtype in ("f16", "bf16", "f32"):
-        for name in ("nf4", "fp4", "dyn8"):
-            code = torch.from_numpy(codebooks.get(name)).to(dev)
-            for bs in (32, 64, 256, 1024, 4096):
-                x = synth.sweep(dtype, bs, seed=1 + ci).to(dev)
-                n = x.numel()
-                a, q = bq.quantize_blockwise(x, code, bs)
-                y = bq.dequantize_blockwise(q, a, n, bs, code, dtype=x.dtype)
-                eb = x.element_size()
-                nbytes = n * eb + q.numel() + 4 * a.numel()
-                tq = _timed(lambda: bq.quantize_blockwise(x, code, bs, absmax=a, out=q), 20, flush)
-                td = _timed(lambda: bq.dequantize_blockwise(q, a, n, bs, code, out=y), 20, flush)
-                cells.append({"dtype": dtype, "codebook": name, "blocksize": bs,
-                              "quantize_us": round(tq * 1e3, 1),
-                              "quantize_gbs": round(nbytes / (tq / 1e3) / 1e9, 1),
-                              "dequantize_us": round(td * 1e3, 1),
-                              "dequantize_gbs": round(nbytes / (td / 1e3) / 1e9, 1)})
-                ci += 1
-    print(json.dumps({"workload": "sweep", "n": synth.SWEEP_N, "cells": cells}), flush=True)
+    """The 45 sweep cells (sweep_cells), one JSON line."""
+    cells, summary = sweep_cells(measured_peaks()[0], reps=max(10, args.steps))
+    print(json.dumps({"workload": "sweep", "n": synth.SWEEP_N, "frac_summary": summary,
+                      "cells": cells}), flush=True)
 
 
 def run_llama(args):
-    """The 224 weight matrices of a Llama-3-8B-shaped model (32 layers),
-    bf16 N(0, 0.02) drawn on the device from a seeded generator per matrix;
-    quantize then dequantize of every matrix back-to-back on one stream."""
-    import dequantization_bq_quantize_b200 as bq
-    dev = torch.device("cuda", torch.cuda.current_device())
-    code = torch.from_numpy(codebooks.nf4()).to(dev)
-    mats, outs = [], []
-    total = 0
-    for layer, i, name, r, c, seed in synth.llama_matrices():
-        g = torch.Generator(device=dev)
-        g.manual_seed(seed)
-        x = torch.randn(r * c, generator=g, device=dev, dtype=torch.float32).mul_(0.02).to(
-            torch.bfloat16)
-        n = x.numel()
-        a = torch.empty((n + BS - 1) // BS, dtype=torch.float32, device=dev)
-        q = torch.empty(n // 2, dtype=torch.uint8, device=dev)
-        y = torch.empty_like(x)
-        mats.append(x)
-        outs.append((a, q, y))
-        total += 2 * quant_bytes(n, BS)
-
-    def everything():
-        for x, (a, q, y) in zip(mats, outs):
-            bq.quantize_blockwise(x, code, BS, absmax=a, out=q)
-            bq.dequantize_blockwise(q, a, x.numel(), BS, code, out=y)
-
-    for _ in range(max(1, args.warmup)):
-        everything()
-    torch.cuda.synchronize()
-    ms_eager = _timed(everything, max(1, args.steps))
-    # the 448 launches captured once in a CUDA graph (the calls allocate
-    # nothing and never synchronise), replayed: device time without host
-    # launch overhead
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(graph, stream=side):
-            everything()
-    torch.cuda.current_stream().wait_stream(side)
-    graph.replay()
-    torch.cuda.synchronize()
-    ms = _timed(graph.replay, max(1, args.steps))
-    print(json.dumps({"workload": "llama3-8b-shaped weight set", "matrices": len(mats),
-                      "eager_ms": round(ms_eager, 3),
-                      "elements": sum(m.numel() for m in mats), "bytes": total,
-                      "ms": round(ms, 3), "gbs": round(total / (ms / 1e3) / 1e9, 1),
-                      "frac_of_measured_peak": round(total / (ms / 1e3) / 1e9 / measured_peaks()[0], 4)}),
-          flush=True)
+    """The Llama-3-8B-shaped weight set (llama_weight_set), one JSON line."""
+    r = llama_weight_set(steps=max(1, args.steps), warmup=max(1, args.warmup))
+    r["frac_of_measured_peak"] = round(r["graph_gbs"] / measured_peaks()[0], 4)
+    print(json.dumps(dict({"workload": "llama3-8b-shaped weight set"}, **r)), flush=True)
 
 
 def run_gguf(args):
