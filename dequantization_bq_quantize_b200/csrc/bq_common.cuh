@@ -255,6 +255,16 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// Orders this thread's earlier generic-proxy accesses to shared memory (plain
+// loads and stores) before later async-proxy accesses to it (bulk / TMA
+// copies).  A consumer that has read a ring stage with plain loads executes it
+// before releasing the stage: the producer's next copy into that stage is an
+// async-proxy write, which the mbarrier release / acquire alone does not order
+// after those loads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Named barrier over `count` threads (a multiple of 32), id != 0.
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

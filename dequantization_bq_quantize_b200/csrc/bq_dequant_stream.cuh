@@ -9,14 +9,21 @@
 // them, decodes and stores, so each iteration's stores wait behind the
 // global-load latency of its own loads: at n = 2^29 bf16 it takes 254 us,
 // and without any loads the same stores take 158 us.  Here the loads run
-// ahead: a persistent grid of 288-thread CTAs, one producer lane streaming
-// each tile's codes (4 KiB for 4-bit, 8 KiB for 8-bit codes of 8192
-// elements) and its slice of absmax into a 4-stage shared-memory ring with
-// 1-D bulk copies (cp.async.bulk, no multicast) completed by mbarrier
-// transaction counts, and 8 consumer warps decoding from shared memory.  A
-// consumer warp owns 128 consecutive 16-byte output chunks of the tile, so
-// its four stores per lane are 2 KiB of contiguous output, and decodes with
-// a per-lane copy of the table (below), free of bank conflicts.
+// ahead: a persistent grid of 544-thread CTAs (3 per SM), one producer lane
+// streaming each tile's codes (4 KiB for 4-bit, 8 KiB for 8-bit codes of
+// 8192 elements) and its slice of absmax into a 4-stage shared-memory ring
+// with 1-D bulk copies (cp.async.bulk, no multicast) completed by mbarrier
+// transaction counts, and 16 consumer warps decoding from shared memory.  A
+// consumer warp owns 64 consecutive 16-byte output chunks of the tile, so its
+// two stores per lane are 1 KiB of contiguous output, and decodes with a
+// per-lane copy of the table (below), free of bank conflicts.  The warps
+// stall on the global store queue: 48 store-issuing warps per SM instead of
+// 32 (8 consumer warps, 4 CTAs per SM) took the kernel in the benchmark step
+// from 237.6 to 232.2 us at n = 2^29.  A consumer releases a stage only after
+// an async-proxy fence: the stage's next fill is a bulk copy, which the
+// mbarrier release / acquire alone does not order after the consumer's plain
+// shared-memory loads (without the fence, a few warps per thousand round
+// trips decoded with the next tile's scales).
 //
 // Used for 4-bit codes with plain statistics when codes, absmax and y are
 // 16-byte aligned and blocksize <= 2048 (so a tile's absmax slice is a whole
@@ -33,7 +40,7 @@ namespace bq {
 
 constexpr int kSTile = 8192;                          // elements per tile
 constexpr int kSStages = 4;
-constexpr int kSConsumerWarps = 8;
+constexpr int kSConsumerWarps = 16;
 constexpr int kSThreads = 32 * (kSConsumerWarps + 1);
 
 // The decode table is replicated per lane so that its lookups never conflict
@@ -126,7 +133,7 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
   }
 
   // consumers: the codebook (pair table for 4-bit codes), then the tiles
-  const int ct = threadIdx.x;  // 0..255
+  const int ct = threadIdx.x;  // 0 .. 32 * kSConsumerWarps - 1
   pdl_wait();
   for (int i = ct; i < E; i += 32 * kSConsumerWarps) s.code[i] = p.code[i];
   if constexpr (NESTED)
@@ -181,6 +188,7 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
         A[u] = s.amax[st][(ch * T::CE) >> p.bs_log2];
       }
     }
+    fence_proxy_async_smem();  // the stage's next fill is an async-proxy write
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp's part is in registers
     const int64_t first = tile * CHUNKS + warp * PER_WARP + lane;

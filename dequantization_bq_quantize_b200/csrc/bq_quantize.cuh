@@ -314,6 +314,7 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
     for (int j = 2; j < kThreadWords; ++j) m2 = amax2<DT>(m2, w[j]);
     amax = max_nan(fabsf(widen_pair_elem<DT>(m2, 0)), fabsf(widen_pair_elem<DT>(m2, 1)));
   }
+  fence_proxy_async_smem();  // the stage's next fill is an async-proxy (TMA) write
   __syncwarp();
   if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
 
