@@ -55,10 +55,11 @@ def _fault(L, reset):
     return v.value
 
 
-# 8 tiles per CTA for either kernel on 148 SMs (quantize: 2 CTAs per SM and
-# 8192 bf16 elements per tile; streaming dequantize: 4 CTAs per SM, 8192
-# elements per tile), so the producer reaches the stage the consumers never
-# freed and its own wait runs out too
+# At least 8 tiles per CTA for either kernel on 148 SMs (quantize: 2 CTAs
+# per SM and 8192 bf16 elements per tile; streaming dequantize: 3 CTAs per
+# SM, 8192 elements per tile), so the producer of the CTA whose tile is
+# skipped reaches the stage its consumers never freed and its own wait runs
+# out too
 N = 4 * 148 * 8 * 8192
 SKIP = 2 * 4 * 148
 
