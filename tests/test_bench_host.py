@@ -6,7 +6,9 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -71,3 +73,45 @@ def test_codebook_option_needs_no_e2e(monkeypatch):
     assert args.codebook == "dyn8" and not args.no_e2e
     with pytest.raises(SystemExit):
         bench.run_ours(args, 0, 1, 0)
+
+
+class _FakeStep:
+    """The attributes bench.verify_step reads, on the CPU, holding outputs
+    computed by the oracle itself (so that they are right by construction)."""
+
+    def __init__(self, n, nblk):
+        import oracle
+        from bq_inputs import codebooks, synth
+        self.codebook = "nf4"
+        self.n = n
+        self.x_cpu, _ = synth.large_outliers(n=n, seed=9, chunk=1 << 14)
+        table = codebooks.nf4()
+        a, q = oracle.quantize_blockwise(synth.to_numpy_bits(self.x_cpu), "bf16", bench.BS, table)
+        y = oracle.dequantize_blockwise(q, a, n, bench.BS, table, "bf16")
+        self.q8_cpu = torch.from_numpy(synth.gguf_blocks(nblk, "q8_0", seed=4).reshape(-1))
+        self.q4_cpu = torch.from_numpy(synth.gguf_blocks(nblk, "q4_0", seed=5).reshape(-1))
+        bf = lambda h: torch.from_numpy(h.view(np.int16)).view(torch.bfloat16)  # noqa: E731
+        self.absmax, self.q, self.y = torch.from_numpy(a), torch.from_numpy(q), bf(y)
+        self.y8 = bf(oracle.dequant_gguf("q8_0", self.q8_cpu.numpy(), "bf16"))
+        self.y4 = bf(oracle.dequant_gguf("q4_0", self.q4_cpu.numpy(), "bf16"))
+
+
+def test_step_verification_accepts_right_and_rejects_any_flipped_bit():
+    """bench.verify_step compares every output bit for bit: the oracle's own
+    outputs pass, and one flipped bit in any of them fails the run."""
+    names = ["quantize", "dequantize", "q8_0", "q4_0"]
+    w = _FakeStep(3 * 8192 + 64 * 5 + 6, 1000)
+    summary, expected = bench.verify_step(w, names, 1)
+    assert summary["ok"] and summary["values_differing"] == 0
+    assert summary["values_compared"] == sum(t.numel() for t in (w.absmax, w.q, w.y, w.y8, w.y4))
+    assert set(expected) == {"absmax", "codes", "dequantize", "q8_0", "q4_0"}
+    for attr in ("absmax", "q", "y", "y8", "y4"):
+        t = getattr(w, attr)
+        raw = t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.uint8)
+        k = raw.numel() // 3
+        raw[k] ^= 1                        # one bit of one value
+        with pytest.raises(RuntimeError, match="differ from the oracle"):
+            bench.verify_step(w, names, 1)
+        raw[k] ^= 1
+    # one-kernel profiling runs are not checked
+    assert bench.verify_step(w, ["quantize"], 1) == (None, None)
