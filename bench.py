@@ -165,9 +165,11 @@ def csrc_digest():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
-    None when the kernel sources changed since those counters were taken."""
+def recorded_traffic(kernel, key="dram_bytes_per_launch"):
+    """Bytes per launch of `kernel` from the committed ncu summary (DRAM read
+    + write by default; key "l2_write_bytes_per_launch" for the bytes the SMs
+    wrote to L2), or None when the kernel sources changed since those
+    counters were taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
@@ -175,8 +177,8 @@ def recorded_traffic(kernel):
         return None
     if t.get("csrc_sha") != csrc_digest():
         return None
-    v = t.get("kernels", {}).get(kernel)
-    return None if v is None else float(v["dram_bytes_per_launch"])
+    v = t.get("kernels", {}).get(kernel, {}).get(key)
+    return None if v is None else float(v)
 
 
 # ---------------------------------------------------------- distributed ----
@@ -670,6 +672,7 @@ def run_ours(args, rank, world, local):
              "q8_0": "gguf_kernel<q8_0,bf16>", "q4_0": "gguf_kernel<q4_0,bf16>"}[dom]
     roof = {"bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak, "unit": "GB/s",
             "frac": kern[dom]["frac"], "traffic": recorded_traffic(kname),
+            "traffic_l2_write": recorded_traffic(kname, "l2_write_bytes_per_launch"),
             "kernel": kname, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"}
 
     cpu = None
