@@ -60,7 +60,7 @@ def parse_args():
                     help="gguf workload: comma-separated types to run (e.g. q4_k,q8_0_encode)")
     ap.add_argument("--gguf-sizes", default="small,matrix",
                     help="gguf workload: 'small' (4096 blocks), 'matrix' (4096 x 14336) or both")
-    ap.add_argument("--workload", choices=["step", "sweep", "llama", "gguf", "nested", "h2d"], default="step",
+    ap.add_argument("--workload", choices=["step", "sweep", "sweep1g", "llama", "gguf", "nested", "h2d"], default="step",
                     help="step: the benchmark line; the others: informational tables")
     return ap.parse_args()
 
@@ -472,6 +472,112 @@ def sweep_cells(peak, reps=10):
     return cells, summary
 
 
+SWEEP_1GIB_TAIL = 37
+
+
+def _block_rows(t, nfull, per_block, sel):
+    """Rows `sel` of the first nfull * per_block values of t, viewed as
+    nfull rows of per_block, brought to the host as raw bits."""
+    return _host_bits(t[: nfull * per_block].view(nfull, per_block)[sel].reshape(-1))
+
+
+def sample_check(x, a, q, y, bs, table, dtype, sample_blocks, threads):
+    """Compare a stratified sample of quantization blocks with the oracle,
+    bit for bit: every (nfull // sample_blocks)-th whole block, the block at
+    element 2^28 (the sweep's zero block, when the input reaches it) and the
+    tail block.  x, a, q, y are the input, absmax, codes and dequantized
+    tensors (any device).  Returns (values compared, values differing,
+    blocks compared)."""
+    import oracle
+    n = x.numel()
+    e = table.size
+    nfull = n // bs
+    stride = max(1, nfull // sample_blocks)
+    sel = set(range(0, nfull, stride))
+    if (1 << 28) // bs < nfull:
+        sel.add((1 << 28) // bs)
+    sel_t = torch.tensor(sorted(sel), dtype=torch.int64, device=x.device)
+    cb = bs // 2 if e == 16 else bs     # code bytes of a whole block
+    xs = np.concatenate([_block_rows(x, nfull, bs, sel_t), _host_bits(x[nfull * bs:])])
+    got = (np.concatenate([_raw_bits(a[sel_t].cpu().numpy()), _raw_bits(a[nfull:].cpu().numpy())]),
+           np.concatenate([_block_rows(q, nfull, cb, sel_t), _host_bits(q[nfull * cb:])]),
+           np.concatenate([_block_rows(y, nfull, bs, sel_t), _host_bits(y[nfull * bs:])]))
+    xin = xs.view(np.float32) if dtype == "f32" else xs
+    oa, oq = oracle.quantize_blockwise_threaded(xin, dtype, bs, table, threads)
+    oy = oracle.dequantize_blockwise_threaded(oq, oa, xs.size, bs, table, dtype, threads)
+    checked = differing = 0
+    for g, exp in zip(got, (oa, oq, oy)):
+        exp = _raw_bits(exp)
+        checked += exp.size
+        differing += int(np.count_nonzero(g != exp)) if g.shape == exp.shape else int(exp.size)
+    return checked, differing, len(sel) + (1 if n % bs else 0)
+
+
+def sweep_1gib(peak, reps=5, sample_blocks=1024):
+    """The sweep at 1 GiB: {fp16, bf16, fp32} x {NF4, FP4, dyn8} x blocksize
+    {32, 64, 256, 1024, 4096}, each cell on n = 2^30 / element size + 37
+    elements (1 GiB of input and a 37-element tail block), N(0, 1) drawn on
+    the device from a generator seeded per dtype, with one all-zero block (the
+    4096 elements from 2^28 on are zero, a whole block at every blocksize).
+    Quantize, and dequantize to the input dtype, each timed with CUDA events
+    (median of `reps` calls; the tensors exceed L2, so no flush).  A
+    stratified sample of each cell's blocks - every (nb // sample_blocks)-th
+    block, the zero block and the tail block - is compared bit for bit with
+    the oracle: absmax, codes and dequantized values."""
+    import dequantization_bq_quantize_b200 as bq
+    import oracle
+    dev = torch.device("cuda", torch.cuda.current_device())
+    threads = oracle.host_threads()
+    cells, checked, differing = [], 0, 0
+    for di, dtype in enumerate(("f16", "bf16", "f32")):
+        tdt = synth.TORCH_DTYPES[dtype]
+        es = torch.empty(0, dtype=tdt).element_size()
+        n = (1 << 30) // es + SWEEP_1GIB_TAIL
+        g = torch.Generator(device=dev)
+        g.manual_seed(200 + di)
+        x = torch.randn(n, generator=g, device=dev, dtype=torch.float32).to(tdt)
+        x[1 << 28: (1 << 28) + 4096] = 0
+        y = torch.empty_like(x)
+        for name in ("nf4", "fp4", "dyn8"):
+            table = codebooks.get(name)
+            code = torch.from_numpy(table).to(dev)
+            e = code.numel()
+            for bs in (32, 64, 256, 1024, 4096):
+                nb = (n + bs - 1) // bs
+                nfull = n // bs
+                a = torch.empty(nb, dtype=torch.float32, device=dev)
+                q = torch.empty((n + 1) // 2 if e == 16 else n, dtype=torch.uint8, device=dev)
+                nbytes = quant_bytes(n, bs, es, e)
+                tq = _event_ms(lambda: bq.quantize_blockwise(x, code, bs, absmax=a, out=q), reps)
+                td = _event_ms(lambda: bq.dequantize_blockwise(q, a, n, bs, code, out=y), reps)
+                c, d, nsel = sample_check(x, a, q, y, bs, table, dtype, sample_blocks, threads)
+                checked += c
+                differing += d
+                cells.append({"dtype": dtype, "codebook": name, "blocksize": bs, "n": n,
+                              "quantize_us": round(tq * 1e3, 1),
+                              "quantize_frac": round(nbytes / (tq / 1e3) / 1e9 / peak, 4),
+                              "dequantize_us": round(td * 1e3, 1),
+                              "dequantize_frac": round(nbytes / (td / 1e3) / 1e9 / peak, 4),
+                              "bytes": nbytes, "blocks_checked": nsel})
+                del a, q
+        del x, y
+    if differing:
+        raise RuntimeError(f"bench: the 1 GiB sweep differs from the oracle in {differing} of "
+                           f"{checked} sampled values")
+    fr = lambda k: sorted(c[k] for c in cells)  # noqa: E731
+    summary = {k: {"min": fr(k)[0], "median": fr(k)[len(cells) // 2], "max": fr(k)[-1]}
+               for k in ("quantize_frac", "dequantize_frac")}
+    return {"n": "2^30 / element size + 37", "l2": "inputs larger than L2; no flush",
+            "frac_summary": summary,
+            "below_0.80": [f"{c['dtype']}/{c['codebook']}/bs{c['blocksize']}/{k[:-5]}"
+                           for c in cells for k in ("quantize_frac", "dequantize_frac")
+                           if c[k] < 0.80],
+            "verified": {"values_compared": checked, "values_differing": differing,
+                         "what": "absmax, codes and dequantized values of a stratified sample of "
+                                 "blocks per cell (about 1024, the zero block and the tail)"},
+            "cells": cells}
+
+
 def llama_weight_set(steps=3, warmup=1):
     """The 224 weight matrices of a Llama-3-8B-shaped model (32 layers), bf16
     N(0, 0.02) drawn on the device from a generator seeded per matrix; NF4
@@ -524,13 +630,14 @@ def llama_weight_set(steps=3, warmup=1):
 
 def run_extras(w):
     """Figures beyond the step, reported next to `value` (not part of it):
-    the 45-cell sweep, the Llama-3-8B-shaped weight set and the 1 GiB
-    quantize / dequantize with the FP4 and dyn8 tables, each against the
-    measured copy bandwidth.  The fault word is checked after them."""
+    the 45-cell sweep at n = 8388645 and at 1 GiB of input per cell, the
+    Llama-3-8B-shaped weight set and the 1 GiB quantize / dequantize with the
+    FP4 and dyn8 tables, each against the measured copy bandwidth.  The fault word is checked after them."""
     peak, kind = measured_peaks()
     t0 = time.perf_counter()
     other = _codebook_figures(w, peak)
     cells, summary = sweep_cells(peak)
+    big = sweep_1gib(peak)
     llama = llama_weight_set()
     llama["graph_frac"] = round(llama["graph_gbs"] / peak, 4)
     llama["eager_frac"] = round(llama["eager_gbs"] / peak, 4)
@@ -541,6 +648,7 @@ def run_extras(w):
     return {"codebooks_1gib": other,
             "sweep": {"n": synth.SWEEP_N, "l2": "flushed (320 MiB read) before every call",
                       "frac_summary": summary, "cells": cells},
+            "sweep_1gib": big,
             "llama_weight_set": llama,
             "extras_peak": f"{peak} GB/s {kind}",
             "extras_seconds": round(time.perf_counter() - t0, 1)}
@@ -921,6 +1029,17 @@ def run_sweep(args):
                       "cells": cells}), flush=True)
 
 
+def run_sweep1g(args):
+    """The 45 sweep cells at 1 GiB of input each (sweep_1gib), one JSON line."""
+    torch.cuda.set_device(0)
+    res = sweep_1gib(measured_peaks()[0], reps=max(5, args.steps))
+    import dequantization_bq_quantize_b200 as bq
+    fault = bq.bq_device_fault(reset=True)
+    if fault:
+        raise SystemExit(f"bench: the fault word was set during the 1 GiB sweep ({fault:#x})")
+    print(json.dumps({"workload": "sweep1g", **res}), flush=True)
+
+
 def run_llama(args):
     """The Llama-3-8B-shaped weight set (llama_weight_set), one JSON line."""
     r = llama_weight_set(steps=max(1, args.steps), warmup=max(1, args.warmup))
@@ -1106,6 +1225,8 @@ def main():
             run_reference(args, rank, world)
         elif args.workload == "sweep":
             run_sweep(args)
+        elif args.workload == "sweep1g":
+            run_sweep1g(args)
         elif args.workload == "llama":
             run_llama(args)
         elif args.workload == "gguf":

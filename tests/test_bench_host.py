@@ -115,3 +115,44 @@ def test_step_verification_accepts_right_and_rejects_any_flipped_bit():
         raw[k] ^= 1
     # one-kernel profiling runs are not checked
     assert bench.verify_step(w, ["quantize"], 1) == (None, None)
+
+
+@pytest.mark.parametrize("dtype,name,bs", [("bf16", "nf4", 64), ("f32", "dyn8", 32),
+                                           ("f16", "fp4", 256)])
+def test_sweep_sample_check_accepts_right_and_rejects_flipped_bits(dtype, name, bs):
+    """bench.sample_check (the 1 GiB sweep's check) compares the sampled
+    blocks and the tail block with the oracle: the oracle's own outputs pass,
+    a flipped bit inside a sampled block or in the tail block is counted, and
+    one in a block outside the sample is not."""
+    import oracle
+    from bq_inputs import codebooks, synth
+    n = 40 * bs + 17                    # 40 whole blocks and a tail block
+    table = codebooks.get(name)
+    x = synth.normal(n, dtype, seed=11)
+    xb = synth.to_numpy_bits(x)
+    a, q = oracle.quantize_blockwise(xb.view(np.float32) if dtype == "f32" else xb, dtype, bs,
+                                     table)
+    y = oracle.dequantize_blockwise(q, a, n, bs, table, dtype)
+    tdt = synth.TORCH_DTYPES[dtype]
+    tt = lambda h: torch.from_numpy(h.view(np.int16 if h.itemsize == 2 else h.dtype)).view(tdt)  # noqa: E731
+    xa, at, qt, yt = x.clone(), torch.from_numpy(a), torch.from_numpy(q), tt(y)
+    # sample every 4th block (40 // 10), so blocks 0, 4, ..., 36 and the tail
+    c, d, nsel = bench.sample_check(xa, at, qt, yt, bs, table, dtype, 10, 2)
+    assert d == 0 and nsel == 11
+    cb = bs // 2 if table.size == 16 else bs
+    assert c == nsel + (10 * cb + (qt.numel() - 40 * cb)) + (10 * bs + 17)
+    raw_y = yt.view(torch.int16) if yt.element_size() == 2 else yt.view(torch.int32)
+    for flip, counted in ((lambda: raw_y.__setitem__(8 * bs + 3, raw_y[8 * bs + 3] ^ 1), True),
+                          (lambda: raw_y.__setitem__(n - 1, raw_y[n - 1] ^ 1), True),
+                          (lambda: raw_y.__setitem__(5 * bs + 3, raw_y[5 * bs + 3] ^ 1), False)):
+        flip()
+        _, d, _ = bench.sample_check(xa, at, qt, yt, bs, table, dtype, 10, 2)
+        assert d == (1 if counted else 0)
+        flip()
+    qt[4 * cb] ^= 1                      # a code byte of sampled block 4
+    _, d, _ = bench.sample_check(xa, at, qt, yt, bs, table, dtype, 10, 2)
+    assert d >= 1
+    qt[4 * cb] ^= 1
+    at[36] = at[36] * 2                 # absmax of sampled block 36
+    _, d, _ = bench.sample_check(xa, at, qt, yt, bs, table, dtype, 10, 2)
+    assert d >= 1
