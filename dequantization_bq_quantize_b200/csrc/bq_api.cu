@@ -135,7 +135,8 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
   auto kernel = bq::quantize_kernel<DT, E, TPB>;
   constexpr size_t smem = bq::qsmem_bytes<E>();
   int occ = 1;
-  bq_status s = kernel_occupancy(slot, kernel, dev, bq::kQThreads, smem, &occ);
+  constexpr int threads = bq::q_threads<TPB>();
+  bq_status s = kernel_occupancy(slot, kernel, dev, threads, smem, &occ);
   if (s != BQ_OK) return s;
   constexpr int BPT = bq::kQConsumers / TPB;
   const int64_t gen_blocks = p.nb - p.full_tiles * BPT;
@@ -145,7 +146,7 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
   if (want < 1) want = 1;
   const int64_t cap = static_cast<int64_t>(occ) * sms;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  cudaError_t e = launch_pdl(kernel, grid, bq::kQThreads, smem, stream, map, p);
+  cudaError_t e = launch_pdl(kernel, grid, threads, smem, stream, map, p);
   return e == cudaSuccess ? BQ_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -204,11 +205,11 @@ bq_status dispatch_dequant(const bq::DParams& p, int entries, int dev, int sms, 
   return launch_dequant<256, OT, NESTED>(p, dev, sms, st);
 }
 
-template <int E, int OT, bool NESTED>
+template <int E, int OT, bool NESTED, bool ADIRECT = false>
 bq_status launch_dequant_stream(const bq::DParams& p, int64_t ntiles, int dev, int sms,
                                 cudaStream_t stream) {
   static KernelSlot slot;
-  auto kernel = bq::dequant_stream_kernel<E, OT, NESTED>;
+  auto kernel = bq::dequant_stream_kernel<E, OT, NESTED, ADIRECT>;
   constexpr size_t smem = bq::ssmem_bytes<E>();
   int occ = 1;
   bq_status s = kernel_occupancy(slot, kernel, dev, bq::kSThreads, smem, &occ);
@@ -239,16 +240,26 @@ bq_status dequant_entry(bq::DParams p, int64_t n, int32_t blocksize, int32_t cod
   // 4-bit codes, 16-byte aligned buffers, at least one whole tile, and a
   // tile's statistics slice a whole number of 16-byte units (plain: 4-byte
   // scales, blocksize <= 2048; nested: 1-byte codes, blocksize <= 512, and
-  // one second-level scale per tile): stream the codes through shared
-  // memory.  (8-bit codes measured faster on dequant_kernel: their 8 KiB
-  // stages and 32-copy table leave 3 CTAs per SM.)
+  // one second-level scale per tile), or plain blocksize 4096 (each warp
+  // reads its one scale): stream the codes through shared memory.  (8-bit
+  // codes measured faster on dequant_kernel: their 8 KiB stages and 32-copy
+  // table leave 3 CTAs per SM.)
   const bool stream_ok =
       NESTED ? (aligned(p.qa, 16) && blocksize <= 512 &&
                 int64_t{blocksize} << p.bs2_log2 >= bq::kSTile)
-             : (aligned(p.absmax, 16) && blocksize <= 2048);
+             : (aligned(p.absmax, 16) || blocksize > 2048);
   if (stream_ok && code_entries == 16 && aligned(p.y, 16) && aligned(p.q, 16) &&
       n >= bq::kSTile) {
     const int64_t ntiles = n / bq::kSTile;
+    if constexpr (!NESTED) {
+      if (blocksize > 2048) {
+        switch (y_dtype) {
+          case BQ_F32: return launch_dequant_stream<16, bq::kF32, false, true>(p, ntiles, dev, info.sms, stream);
+          case BQ_F16: return launch_dequant_stream<16, bq::kF16, false, true>(p, ntiles, dev, info.sms, stream);
+          default: return launch_dequant_stream<16, bq::kBF16, false, true>(p, ntiles, dev, info.sms, stream);
+        }
+      }
+    }
     switch (y_dtype) {
       case BQ_F32: return launch_dequant_stream<16, bq::kF32, NESTED>(p, ntiles, dev, info.sms, stream);
       case BQ_F16: return launch_dequant_stream<16, bq::kF16, NESTED>(p, ntiles, dev, info.sms, stream);

@@ -26,12 +26,13 @@
 // trips decoded with the next tile's scales).
 //
 // Used for 4-bit codes with plain statistics when codes, absmax and y are
-// 16-byte aligned and blocksize <= 2048 (so a tile's absmax slice is a whole
-// number of 16-byte units); the elements after the last whole tile are done
-// one per thread from global memory.  (The template also covers 8-bit codes,
-// which measured faster on dequant_kernel.)  Every mbarrier wait gives up after a bounded time,
-// sets a bit of the device fault word (4: consumer, 8: producer) and leaves
-// the kernel instead of hanging.
+// 16-byte aligned: blocksize <= 2048 streams the tile's absmax slice (a whole
+// number of 16-byte units) with the codes, blocksize 4096 has each warp read
+// its one scale directly (ADIRECT); the elements after the last whole tile are
+// done one per thread from global memory.  (The template also covers 8-bit
+// codes, which measured faster on dequant_kernel.)  Every mbarrier wait gives
+// up after a bounded time, sets a bit of the device fault word (4: consumer,
+// 8: producer) and leaves the kernel instead of hanging.
 #pragma once
 
 #include "bq_dequant.cuh"
@@ -79,8 +80,14 @@ __device__ __forceinline__ uint2 smem_codes(const uint8_t* base, int chunk) {
 // (blocksize * blocksize2 >= the tile, so one per tile) comes from global
 // memory, fetched a tile ahead.  A_b = RN(code2[qa_b] * absmax2), as in
 // dequant_kernel.
-template <int E, int OT, bool NESTED>
+//
+// ADIRECT (plain statistics, blocksize 4096: a tile's two scales are 8 bytes,
+// not a whole 16-byte unit): the ring carries only codes, and each consumer
+// warp reads the one scale of its 512 outputs (a warp's part of a tile lies in
+// one block when blocksize >= 512) from global memory, a tile ahead.
+template <int E, int OT, bool NESTED, bool ADIRECT = false>
 __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams p, int64_t ntiles) {
+  static_assert(!(NESTED && ADIRECT), "one statistics form");
   using T = DTraits<E, OT>;
   constexpr int CHUNKS = kSTile / T::CE;                 // 16-byte output chunks per tile
   constexpr int PER_WARP = CHUNKS / kSConsumerWarps;     // 128 or 256
@@ -117,12 +124,13 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
           }
         }
         if (test_skip_tile(tile)) continue;  // fault-path test builds only
-        const uint32_t abytes = (NESTED ? 1u : 4u) * static_cast<uint32_t>(abs_per_tile);
+        const uint32_t abytes =
+            ADIRECT ? 0u : (NESTED ? 1u : 4u) * static_cast<uint32_t>(abs_per_tile);
         mbar_arrive_expect_tx(&s.full[st], CODE_BYTES + abytes);
         bulk_load(s.codes[st], p.q + tile * CODE_BYTES, CODE_BYTES, &s.full[st], pol);
         if constexpr (NESTED)
           bulk_load(s.amax[st], p.qa + tile * abs_per_tile, abytes, &s.full[st], pol);
-        else
+        else if constexpr (!ADIRECT)
           bulk_load(s.amax[st], p.absmax + tile * abs_per_tile, abytes, &s.full[st], pol);
       }
       // every copy issued must have landed before the CTA may exit
@@ -156,17 +164,27 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
   // NESTED: second-level scale of the tile (block index >> bs2_log2 of the
   // tile's first block), loaded one tile ahead
   const int sh2 = p.bs2_log2 + p.bs_log2;
-  float a2_next = 0.0f;
+  // ADIRECT: the scale of this warp's 512 outputs, likewise a tile ahead
+  const int64_t wofs = static_cast<int64_t>(warp) * (kSTile / kSConsumerWarps);
+  float a2_next = 0.0f, aw_next = 0.0f;
   if constexpr (NESTED)
     if (static_cast<int64_t>(blockIdx.x) < ntiles)
       a2_next = __ldg(p.absmax2 + ((static_cast<int64_t>(blockIdx.x) * kSTile) >> sh2));
+  if constexpr (ADIRECT)
+    if (static_cast<int64_t>(blockIdx.x) < ntiles)
+      aw_next = __ldg(p.absmax + ((static_cast<int64_t>(blockIdx.x) * kSTile + wofs) >> p.bs_log2));
   int64_t iter = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
-    float a2 = 0.0f;
+    float a2 = 0.0f, aw = 0.0f;
     if constexpr (NESTED) {
       a2 = a2_next;
       const int64_t nt = tile + gridDim.x;
       if (nt < ntiles) a2_next = __ldg(p.absmax2 + ((nt * kSTile) >> sh2));
+    }
+    if constexpr (ADIRECT) {
+      aw = aw_next;
+      const int64_t nt = tile + gridDim.x;
+      if (nt < ntiles) aw_next = __ldg(p.absmax + ((nt * kSTile + wofs) >> p.bs_log2));
     }
     const int st = static_cast<int>(iter % kSStages);
     // warp-uniform: if any lane gives up, the whole warp leaves together
@@ -184,6 +202,8 @@ __global__ void __launch_bounds__(kSThreads) dequant_stream_kernel(const DParams
       if constexpr (NESTED) {
         const uint32_t qa = reinterpret_cast<const uint8_t*>(s.amax[st])[(ch * T::CE) >> p.bs_log2];
         A[u] = __fmul_rn(s.code2[qa], a2);
+      } else if constexpr (ADIRECT) {
+        A[u] = aw;
       } else {
         A[u] = s.amax[st][(ch * T::CE) >> p.bs_log2];
       }

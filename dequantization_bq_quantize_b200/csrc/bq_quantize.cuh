@@ -6,14 +6,16 @@
 // (lowest index on ties), codes packed two per byte high nibble first
 // (16-entry tables) or one per byte (256-entry tables).
 //
-// Kernel design.  A persistent grid (2 CTAs per SM) of 288-thread CTAs: one
-// producer warp streams 16 KiB input tiles (128 rows of 128 B) into a 4-stage
+// Kernel design.  A persistent grid (2 CTAs per SM) of 288-thread CTAs (320
+// with the statistics warp): one producer warp streams 16 KiB input tiles (128 rows of 128 B) into a 4-stage
 // shared-memory ring with 2-D TMA loads (128-byte swizzle, no multicast), and
 // 8 consumer warps process each tile.  Consumer thread t owns 64 contiguous
 // bytes (row t/2, half t%2), read with four conflict-free 16-byte shared
 // loads thanks to the swizzle.  A quantization block spans TPB =
 // blocksize * elem_bytes / 64 consecutive threads: its absmax is a shuffle-xor
-// tree over TPB lanes, plus a shared-memory step across warps when TPB > 32.
+// tree over TPB lanes (one integer warp reduction when TPB = 32); blocks
+// wider than a warp (TPB > 32) get theirs from a statistics warp that reads
+// each tile as it lands (stats_main), so no consumer warp waits for another.
 // The stage is released as soon as the values are in registers.
 //
 // Per element the fast path costs about ten instructions:
@@ -44,7 +46,6 @@ namespace bq {
 
 constexpr int kQConsumerWarps = 8;
 constexpr int kQConsumers = kQConsumerWarps * 32;  // 256
-constexpr int kQThreads = kQConsumers + 32;        // + producer warp
 constexpr int kTileBytes = 16384;
 constexpr int kTileRows = 128;                     // rows of 128 bytes
 constexpr int kStages = 4;
@@ -52,13 +53,24 @@ constexpr int kThreadBytes = kTileBytes / kQConsumers;  // 64
 constexpr int kThreadWords = kThreadBytes / 4;           // 16
 static_assert(kThreadBytes == 64, "thread owns four 16-byte chunks");
 
+// Blocks that span more than one warp of consumers (TPB > 32 threads) get
+// their absmax from a statistics warp instead of a reduction across the
+// consumer warps: the statistics warp reads each tile as it lands, writes the
+// absmax of its blocks to shared memory and signals an mbarrier, so the
+// consumer warps never wait for one another (a cross-warp reduction put a
+// CTA-wide barrier on every tile: bf16 blocksize 4096 ran at 0.72-0.76 of the
+// measured copy bandwidth against 0.89-0.99 for smaller blocks).
+template <int TPB> constexpr bool kStatsWarp = TPB > 32;
+template <int TPB> constexpr int q_threads() { return kQConsumers + (kStatsWarp<TPB> ? 64 : 32); }
+constexpr int kQMaxTileBlocks = 4;   // blocks per tile when TPB > 32 (TPB >= 64)
+
 template <int E>
 struct QSmem {
   uint8_t stage[kStages][kTileBytes];  // 1024-byte aligned (128B swizzle)
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  float red[2][kQConsumerWarps];
-  int cabort[2];   // per tile-iteration parity: a consumer gave up waiting
+  uint64_t stats[kStages];             // statistics warp: the stage's absmax is ready
+  float tamax[kStages][kQMaxTileBlocks];
   TableSmem tab;
   Lut<E> lut;
 };
@@ -276,17 +288,16 @@ __device__ __forceinline__ void encode_safe(const uint32_t (&w)[kThreadWords], c
 
 template <int DT, int E, int TPB, int MODE, bool REMAP>
 __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uint32_t tile,
-                                              int st, uint32_t par, uint32_t iter, int ct,
-                                              uint32_t t_base) {
+                                              int st, uint32_t par, int ct, uint32_t t_base) {
   using O = QOut<DT, E>;
   constexpr int TE = kTileBytes / ElemBytes<DT>::value;
   constexpr int BPT = kQConsumers / TPB;
-  const int lane = ct & 31, cw = ct >> 5;
+  const int lane = ct & 31;
 
-  const bool ok = mbar_wait_bounded(&s.full[st], par);
-  if (!ok) {
+  // warp-uniform: if any lane gives up, the whole warp leaves together
+  if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s.full[st], par))) {
     if (lane == 0) record_fault(1u);
-    s.cabort[iter & 1] = 1;
+    return false;
   }
 
   // four 16-byte chunks of row ct/2, physical chunk = logical ^ (row % 8)
@@ -302,46 +313,46 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
     }
   }
 
-  // thread-local absmax, NaN-propagating
-  float amax;
-  if constexpr (DT == kF32) {
-    amax = fabsf(__uint_as_float(w[0]));
-#pragma unroll
-    for (int j = 1; j < kThreadWords; ++j) amax = max_nan(amax, fabsf(__uint_as_float(w[j])));
+  float A;
+  if constexpr (kStatsWarp<TPB>) {
+    // the statistics warp's absmax of this thread's block
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s.stats[st], par))) {
+      if (lane == 0) record_fault(1u);
+      return false;
+    }
+    A = s.tamax[st][ct / TPB];
+    fence_proxy_async_smem();  // the stage's next fill is an async-proxy (TMA) write
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
   } else {
-    uint32_t m2 = amax2<DT>(w[0], w[1]);
+    // thread-local absmax, NaN-propagating
+    float amax;
+    if constexpr (DT == kF32) {
+      amax = fabsf(__uint_as_float(w[0]));
 #pragma unroll
-    for (int j = 2; j < kThreadWords; ++j) m2 = amax2<DT>(m2, w[j]);
-    amax = max_nan(fabsf(widen_pair_elem<DT>(m2, 0)), fabsf(widen_pair_elem<DT>(m2, 1)));
-  }
-  fence_proxy_async_smem();  // the stage's next fill is an async-proxy (TMA) write
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
+      for (int j = 1; j < kThreadWords; ++j) amax = max_nan(amax, fabsf(__uint_as_float(w[j])));
+    } else {
+      uint32_t m2 = amax2<DT>(w[0], w[1]);
+#pragma unroll
+      for (int j = 2; j < kThreadWords; ++j) m2 = amax2<DT>(m2, w[j]);
+      amax = max_nan(fabsf(widen_pair_elem<DT>(m2, 0)), fabsf(widen_pair_elem<DT>(m2, 1)));
+    }
+    fence_proxy_async_smem();  // the stage's next fill is an async-proxy (TMA) write
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
 
-  bool abort_now = !ok;
-  float m = amax;
-  if constexpr (TPB > 1 && TPB <= 32) {
+    float m = amax;
+    if constexpr (TPB == 32) {
+      // |x| >= 0 (or a NaN with the sign clear): the bits order as unsigned
+      // integers, NaN above +inf, so one integer max reduces the warp
+      m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+    } else if constexpr (TPB > 1) {
 #pragma unroll
-    for (int off = 1; off < TPB; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
-  } else if constexpr (TPB > 32) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
-    constexpr int WPB = TPB / 32;
-    const int pb = static_cast<int>(iter & 1);
-    if (lane == 0) s.red[pb][cw] = m;
-    named_sync(1, kQConsumers);
-    const int g0 = (cw / WPB) * WPB;
-    m = s.red[pb][g0];
-#pragma unroll
-    for (int i = 1; i < WPB; ++i) m = max_nan(m, s.red[pb][g0 + i]);
-    // set before this barrier by any warp that gave up on this tile; the slot
-    // of the other parity may already be written by a warp one tile ahead
-    abort_now = *reinterpret_cast<volatile int*>(&s.cabort[iter & 1]) != 0;
+      for (int off = 1; off < TPB; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
+    }
+    A = m;
+    if (ct % TPB == 0) p.absmax[static_cast<int64_t>(tile) * BPT + ct / TPB] = A;
   }
-  const float A = m;
-  if (abort_now) return false;
-
-  if (ct % TPB == 0) p.absmax[static_cast<int64_t>(tile) * BPT + ct / TPB] = A;
 
   uint32_t ow[O::NW];
   // bucket path: the block's reciprocal is valid for Markstein's form (the
@@ -391,6 +402,69 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
   }
 }
 
+// ---------------------------------------------------- statistics warp ----
+
+// Absmax of every quantization block of each tile (TPB > 32: a block is
+// TPB / 2 >= 32 whole 128-byte rows, one to four blocks per tile), written to
+// the stage's tamax slots and to global memory; then the stage's stats
+// mbarrier is signalled and the stage released like a consumer warp does.
+// Step k reads bytes [512 k, 512 k + 512) of the stage, lane l the 16 bytes at
+// 512 k + 16 l (four whole rows, so the 128-byte swizzle, a permutation within
+// each row, does not matter, and the warp's load is free of bank conflicts);
+// a block is TPB / 8 consecutive steps.  |x| is kept as bits: for values >= 0
+// (and NaN, sign cleared) the unsigned order is the float order with NaN above
+// +inf, so the warp's maximum is one integer reduction.
+template <int DT, int E, int TPB>
+__device__ void stats_main(QSmem<E>& s, const QParams& p, int lane) {
+  constexpr int BPT = kQConsumers / TPB;
+  constexpr int STEPS = TPB / 8;   // 512-byte steps per block
+  static_assert(BPT <= kQMaxTileBlocks && STEPS * BPT == kTileBytes / 512, "tile split");
+  pdl_wait();  // absmax is written to global memory
+  const uint32_t ntiles = static_cast<uint32_t>(p.full_tiles);
+  uint32_t iter = 0;
+  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
+    const int st = static_cast<int>(iter % kStages);
+    const uint32_t par = (iter / kStages) & 1u;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s.full[st], par))) {
+      if (lane == 0) record_fault(1u);
+      break;
+    }
+    const uint8_t* src = s.stage[st] + 16 * lane;
+#pragma unroll
+    for (int b = 0; b < BPT; ++b) {
+      uint32_t mb;  // bits of this lane's max |x| over the block
+      if constexpr (DT == kF32) {
+        float m = 0.0f;
+#pragma unroll 8
+        for (int k = 0; k < STEPS; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + 512 * (b * STEPS + k));
+          m = max_nan(m, max_nan(max_nan(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                                 max_nan(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
+        }
+        mb = __float_as_uint(m);
+      } else {
+        uint32_t m2 = 0u;
+#pragma unroll 8
+        for (int k = 0; k < STEPS; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + 512 * (b * STEPS + k));
+          m2 = amax2<DT>(m2, amax2<DT>(amax2<DT>(v.x, v.y), amax2<DT>(v.z, v.w)));
+        }
+        mb = __float_as_uint(max_nan(fabsf(widen_pair_elem<DT>(m2, 0)),
+                                     fabsf(widen_pair_elem<DT>(m2, 1))));
+      }
+      const float A = __uint_as_float(__reduce_max_sync(0xffffffffu, mb));
+      if (lane == 0) {
+        s.tamax[st][b] = A;
+        p.absmax[static_cast<int64_t>(tile) * BPT + b] = A;
+      }
+    }
+    if (lane == 0) mbar_arrive(&s.stats[st]);  // releases the tamax writes
+    fence_proxy_async_smem();  // the stage's next fill is an async-proxy (TMA) write
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[st]);
+  }
+}
+
 // ------------------------------------------------------------- kernel -----
 
 template <int DT, int E, int TPB, int MODE, bool REMAP = false>
@@ -402,7 +476,7 @@ __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
     const int st = static_cast<int>(iter % kStages);
     const uint32_t par = (iter / kStages) & 1u;
-    if (!quantize_tile<DT, E, TPB, MODE, REMAP>(s, p, tile, st, par, iter, ct, t_base)) break;
+    if (!quantize_tile<DT, E, TPB, MODE, REMAP>(s, p, tile, st, par, ct, t_base)) break;
   }
   // what the tiles did not cover: one quantization block per warp
   const int lane = ct & 31, cw = ct >> 5;
@@ -413,20 +487,20 @@ __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int
 }
 
 template <int DT, int E, int TPB>
-__global__ void __launch_bounds__(kQThreads, 2)
+__global__ void __launch_bounds__(q_threads<TPB>(), 2)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap, const QParams p) {
   extern __shared__ uint8_t smem_raw[];
   QSmem<E>& s = *reinterpret_cast<QSmem<E>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr bool SW = kStatsWarp<TPB>;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kQConsumerWarps);
+      mbar_init(&s.empty[i], kQConsumerWarps + (SW ? 1 : 0));
+      mbar_init(&s.stats[i], 1);
     }
-    s.cabort[0] = 0;
-    s.cabort[1] = 0;
     fence_mbar_init();
   }
   pdl_release();
@@ -461,8 +535,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
     }
     return;
   }
+  if constexpr (SW) {
+    if (warp == 1) {
+      stats_main<DT, E, TPB>(s, p, lane);
+      return;
+    }
+  }
 
-  const int ct = threadIdx.x - 32;
+  const int ct = threadIdx.x - (SW ? 64 : 32);
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   pdl_wait();
   // the tables stand only if the codebook, read at L2 after the wait, still

@@ -393,6 +393,20 @@ def test_config_sweep_full(dtype, name):
         _run_full(x, dtype, bs, name)
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("name", ["nf4", "dyn8"])
+def test_wide_blocks_ring_wrap_full(dtype, name):
+    """Blocks wider than a warp of quantize threads (fp16 / bf16 blocksize
+    2048 and 4096, fp32 blocksize 1024 to 4096: absmax from the statistics
+    warp) and the streaming dequantization's blocksize-4096 form (each warp
+    reads its scale), at n = 2^25 + 37: about 14 tiles per CTA, so every ring
+    and its mbarrier phases wrap several times.  Every output against the
+    oracle."""
+    for i, bs in enumerate((1024, 2048, 4096)):
+        x = synth.sweep(dtype, bs, seed=500 + i, n=(1 << 25) + 37)
+        _run_full(x, dtype, bs, name)
+
+
 def test_config_large_bf16_nf4_full():
     """bf16 n = 2^29 (1 GiB) N(0, 0.02) with 0.1% outliers, NF4, blocksize 64:
     every output (the persistent rings wrap hundreds of times per CTA)."""
