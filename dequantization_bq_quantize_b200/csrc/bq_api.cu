@@ -237,34 +237,32 @@ bq_status dequant_entry(bq::DParams p, int64_t n, int32_t blocksize, int32_t cod
   const int qb = code_entries == 16 ? ce / 2 : ce;
   p.vec = aligned(p.y, 16) && aligned(p.q, qb);
   p.nchunks = p.vec ? n / ce : 0;
-  // 4-bit codes, 16-byte aligned buffers, at least one whole tile, and a
-  // tile's statistics slice a whole number of 16-byte units (plain: 4-byte
-  // scales, blocksize <= 2048; nested: 1-byte codes, blocksize <= 512, and
-  // one second-level scale per tile), or plain blocksize 4096 (each warp
-  // reads its one scale): stream the codes through shared memory.  (8-bit
-  // codes measured faster on dequant_kernel: their 8 KiB stages and 32-copy
-  // table leave 3 CTAs per SM.)
+  // 4-bit codes, 16-byte aligned buffers, 16-bit outputs, at least one whole
+  // tile, and a tile's statistics slice a whole number of 16-byte units
+  // (plain: 4-byte scales, blocksize <= 2048; nested: 1-byte codes,
+  // blocksize <= 512, and one second-level scale per tile), or plain
+  // blocksize 4096 (each warp reads its one scale): stream the codes through
+  // shared memory.  (8-bit codes measured faster on dequant_kernel: their
+  // 8 KiB stages and 32-copy table leave 3 CTAs per SM.  So did fp32
+  // outputs, whose stores are twice as many per code byte: 1 GiB fp32 NF4,
+  // 207-211 us against 214-222 us streamed.)
   const bool stream_ok =
       NESTED ? (aligned(p.qa, 16) && blocksize <= 512 &&
                 int64_t{blocksize} << p.bs2_log2 >= bq::kSTile)
              : (aligned(p.absmax, 16) || blocksize > 2048);
   if (stream_ok && code_entries == 16 && aligned(p.y, 16) && aligned(p.q, 16) &&
-      n >= bq::kSTile) {
+      y_dtype != BQ_F32 && n >= bq::kSTile) {
     const int64_t ntiles = n / bq::kSTile;
     if constexpr (!NESTED) {
       if (blocksize > 2048) {
-        switch (y_dtype) {
-          case BQ_F32: return launch_dequant_stream<16, bq::kF32, false, true>(p, ntiles, dev, info.sms, stream);
-          case BQ_F16: return launch_dequant_stream<16, bq::kF16, false, true>(p, ntiles, dev, info.sms, stream);
-          default: return launch_dequant_stream<16, bq::kBF16, false, true>(p, ntiles, dev, info.sms, stream);
-        }
+        if (y_dtype == BQ_F16)
+          return launch_dequant_stream<16, bq::kF16, false, true>(p, ntiles, dev, info.sms, stream);
+        return launch_dequant_stream<16, bq::kBF16, false, true>(p, ntiles, dev, info.sms, stream);
       }
     }
-    switch (y_dtype) {
-      case BQ_F32: return launch_dequant_stream<16, bq::kF32, NESTED>(p, ntiles, dev, info.sms, stream);
-      case BQ_F16: return launch_dequant_stream<16, bq::kF16, NESTED>(p, ntiles, dev, info.sms, stream);
-      default: return launch_dequant_stream<16, bq::kBF16, NESTED>(p, ntiles, dev, info.sms, stream);
-    }
+    if (y_dtype == BQ_F16)
+      return launch_dequant_stream<16, bq::kF16, NESTED>(p, ntiles, dev, info.sms, stream);
+    return launch_dequant_stream<16, bq::kBF16, NESTED>(p, ntiles, dev, info.sms, stream);
   }
   switch (y_dtype) {
     case BQ_F32: return dispatch_dequant<bq::kF32, NESTED>(p, code_entries, dev, info.sms, stream);

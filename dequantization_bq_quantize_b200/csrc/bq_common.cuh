@@ -50,9 +50,16 @@ __device__ __forceinline__ float widen_pair_elem<kBF16>(uint32_t w, int hi) {
   return __uint_as_float(hi ? (w & 0xffff0000u) : (w << 16));
 }
 
+// fp16 -> fp32 as the mixed-precision add h + (-0.0) (fp16 operand, fp32
+// result): exact, with -0 + -0 = -0 and +0 + -0 = +0, and issued on the FMA
+// pipe.  The plain conversion measured slower where the kernels widen every
+// element (fp16 NF4 blocksize 64 quantize of 1 GiB: 236.0 -> 219.6 us).
 template <>
 __device__ __forceinline__ float widen_pair_elem<kF16>(uint32_t w, int hi) {
-  return __half2float(__ushort_as_half((unsigned short)(hi ? (w >> 16) : (w & 0xffffu))));
+  float d;
+  const unsigned short h = static_cast<unsigned short>(hi ? (w >> 16) : (w & 0xffffu));
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(h), "f"(-0.0f));
+  return d;
 }
 
 // Scalar element load from global memory (any alignment of the element type).
