@@ -241,11 +241,11 @@ bq_status dequant_entry(bq::DParams p, int64_t n, int32_t blocksize, int32_t cod
   // tile, and a tile's statistics slice a whole number of 16-byte units
   // (plain: 4-byte scales, blocksize <= 2048; nested: 1-byte codes,
   // blocksize <= 512, and one second-level scale per tile), or plain
-  // blocksize 4096 (each warp reads its one scale): stream the codes through
-  // shared memory.  (8-bit codes measured faster on dequant_kernel: their
-  // 8 KiB stages and 32-copy table leave 3 CTAs per SM.  So did fp32
-  // outputs, whose stores are twice as many per code byte: 1 GiB fp32 NF4,
-  // 207-211 us against 214-222 us streamed.)
+  // blocksize 4096 (the producer copies the tile's two scales): stream the
+  // codes through shared memory.  (8-bit codes measured faster on
+  // dequant_kernel: their 8 KiB stages and 32-copy table leave 3 CTAs per
+  // SM.  So did fp32 outputs, whose stores are twice as many per code byte:
+  // 1 GiB fp32 NF4, 207-211 us against 214-222 us streamed.)
   const bool stream_ok =
       NESTED ? (aligned(p.qa, 16) && blocksize <= 512 &&
                 int64_t{blocksize} << p.bs2_log2 >= bq::kSTile)
