@@ -135,7 +135,7 @@ bq_status launch_quantize(const bq::QParams& p, const CUtensorMap& map, int dev,
   auto kernel = bq::quantize_kernel<DT, E, TPB>;
   constexpr size_t smem = bq::qsmem_bytes<E>();
   int occ = 1;
-  constexpr int threads = bq::q_threads<TPB>();
+  constexpr int threads = bq::q_threads<DT, E, TPB>();
   bq_status s = kernel_occupancy(slot, kernel, dev, threads, smem, &occ);
   if (s != BQ_OK) return s;
   constexpr int BPT = bq::kQConsumers / TPB;

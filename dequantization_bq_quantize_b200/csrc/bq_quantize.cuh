@@ -61,7 +61,17 @@ static_assert(kThreadBytes == 64, "thread owns four 16-byte chunks");
 // CTA-wide barrier on every tile: bf16 blocksize 4096 ran at 0.72-0.76 of the
 // measured copy bandwidth against 0.89-0.99 for smaller blocks).
 template <int TPB> constexpr bool kStatsWarp = TPB > 32;
-template <int TPB> constexpr int q_threads() { return kQConsumers + (kStatsWarp<TPB> ? 64 : 32); }
+// 16-bit inputs with 16-entry tables (two or four blocks per tile) split the
+// statistics work over two warps, block b to warp b % 2: one statistics warp
+// adds its ~170 instructions per tile to a single SM sub-partition, which
+// then limits the issue-bound kernel (bf16 NF4 blocksize 4096, 1 GiB:
+// 258.4 -> 252.4 us).  256-entry tables keep one (their consumers need 96
+// registers; 352-thread CTAs at two per SM allow 88), and fp32 inputs,
+// which leave issue slots to spare, keep one.
+template <int DT, int E, int TPB>
+constexpr int kNumStats = TPB > 32 ? ((DT != kF32 && E == 16) ? 2 : 1) : 0;
+template <int DT, int E, int TPB>
+constexpr int q_threads() { return kQConsumers + 32 + 32 * kNumStats<DT, E, TPB>; }
 constexpr int kQMaxTileBlocks = 4;   // blocks per tile when TPB > 32 (TPB >= 64)
 
 template <int E>
@@ -404,10 +414,11 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 
 // ---------------------------------------------------- statistics warp ----
 
-// Absmax of every quantization block of each tile (TPB > 32: a block is
-// TPB / 2 >= 32 whole 128-byte rows, one to four blocks per tile), written to
-// the stage's tamax slots and to global memory; then the stage's stats
-// mbarrier is signalled and the stage released like a consumer warp does.
+// Absmax of the quantization blocks b of each tile with b % NSW == sw (TPB >
+// 32: a block is TPB / 2 >= 32 whole 128-byte rows, one to four blocks per
+// tile), written to the stage's tamax slots and to global memory; then the
+// stage's stats mbarrier (NSW arrivals) is signalled and the stage released
+// like a consumer warp does.
 // Step k reads bytes [512 k, 512 k + 512) of the stage, lane l the 16 bytes at
 // 512 k + 16 l (four whole rows, so the 128-byte swizzle, a permutation within
 // each row, does not matter, and the warp's load is free of bank conflicts);
@@ -415,7 +426,8 @@ __device__ void quantize_block_generic(const QParams& p, const QSmem<E>& s, int6
 // (and NaN, sign cleared) the unsigned order is the float order with NaN above
 // +inf, so the warp's maximum is one integer reduction.
 template <int DT, int E, int TPB>
-__device__ void stats_main(QSmem<E>& s, const QParams& p, int lane) {
+__device__ void stats_main(QSmem<E>& s, const QParams& p, int lane, int sw) {
+  constexpr int NSW = kNumStats<DT, E, TPB>;
   constexpr int BPT = kQConsumers / TPB;
   constexpr int STEPS = TPB / 8;   // 512-byte steps per block
   static_assert(BPT <= kQMaxTileBlocks && STEPS * BPT == kTileBytes / 512, "tile split");
@@ -432,6 +444,7 @@ __device__ void stats_main(QSmem<E>& s, const QParams& p, int lane) {
     const uint8_t* src = s.stage[st] + 16 * lane;
 #pragma unroll
     for (int b = 0; b < BPT; ++b) {
+      if (b % NSW != sw) continue;
       uint32_t mb;  // bits of this lane's max |x| over the block
       if constexpr (DT == kF32) {
         float m = 0.0f;
@@ -487,19 +500,20 @@ __device__ __forceinline__ void consumer_main(QSmem<E>& s, const QParams& p, int
 }
 
 template <int DT, int E, int TPB>
-__global__ void __launch_bounds__(q_threads<TPB>(), 2)
+__global__ void __launch_bounds__(q_threads<DT, E, TPB>(), 2)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap, const QParams p) {
   extern __shared__ uint8_t smem_raw[];
   QSmem<E>& s = *reinterpret_cast<QSmem<E>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool SW = kStatsWarp<TPB>;
+  constexpr int NSW = kNumStats<DT, E, TPB>;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kQConsumerWarps + (SW ? 1 : 0));
-      mbar_init(&s.stats[i], 1);
+      mbar_init(&s.empty[i], kQConsumerWarps + NSW);
+      mbar_init(&s.stats[i], NSW > 0 ? NSW : 1);
     }
     fence_mbar_init();
   }
@@ -536,13 +550,13 @@ __global__ void __launch_bounds__(q_threads<TPB>(), 2)
     return;
   }
   if constexpr (SW) {
-    if (warp == 1) {
-      stats_main<DT, E, TPB>(s, p, lane);
+    if (warp >= 1 && warp <= NSW) {
+      stats_main<DT, E, TPB>(s, p, lane, warp - 1);
       return;
     }
   }
 
-  const int ct = threadIdx.x - (SW ? 64 : 32);
+  const int ct = threadIdx.x - 32 * (1 + NSW);
   build_search<E, kQConsumers>(s.tab, s.lut, p.code, ct);
   pdl_wait();
   // the tables stand only if the codebook, read at L2 after the wait, still
