@@ -207,13 +207,15 @@ __device__ __forceinline__ constexpr float half_weight(int j) {
 //             bytes are merged with one byte permute per word.
 //  kModeLutI (256-entry tables): code = byte 2 of i[b] + key(q)
 //             (bq_search.cuh); byte permutes gather four codes into a word.
+//  PREW: the elements come already widened to fp32 in xe (quantize_tile).
 //  REMAP (16-entry tables like FP4, whose +-0 pair makes one step of two):
 //             the table holds ranks of the distinct values, which step by
 //             one; each nibble >= 8 then gets 1 added (ranks 8..14 -> codes
 //             9..15), three instructions per 8 codes.
-template <int DT, int E, int MODE, bool REMAP>
+template <int DT, int E, int MODE, bool REMAP, bool PREW = false>
 __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], const BlockScale& sc,
-                                            uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW]) {
+                                            uint32_t t_base, uint32_t (&ow)[QOut<DT, E>::NW],
+                                            const float* xe = nullptr) {
   using O = QOut<DT, E>;
   constexpr int NH = 2 * O::NW;                 // 16-bit halves
   constexpr int PER_HALF = O::EPT / NH;         // elements per half (4 or 2)
@@ -227,7 +229,8 @@ __device__ __forceinline__ void encode_fast(const uint32_t (&w)[kThreadWords], c
     if constexpr (DT == kF32)
       div_fast2(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
     else
-      div_fast2_2term(tile_elem<DT>(w, 2 * i), tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
+      div_fast2_2term(PREW ? xe[2 * i] : tile_elem<DT>(w, 2 * i),
+                      PREW ? xe[2 * i + 1] : tile_elem<DT>(w, 2 * i + 1), sc, q0, q1);
     if constexpr (MODE == kModeLutI) {
       static_assert(E == 256, "integer select is built for 256-entry tables only");
       pair[i] = __byte_perm(lut_int_sum(q0, t_base), lut_int_sum(q1, t_base), 0x0062);
@@ -324,6 +327,12 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   }
 
   float A;
+  // 16-bit inputs, blocks of 4 to 16 threads: widen the elements to fp32
+  // before the shuffle tree, so that the compiler can place that independent
+  // work between the tree's dependent steps (bf16 / fp16 NF4 blocksize 256,
+  // 1 GiB: 229.8 -> 225.6 / 221.4 us; blocks of 2 threads gained nothing)
+  constexpr bool PREW_T = DT != kF32 && TPB >= 4 && TPB < 32;
+  float xe[O::EPT];
   if constexpr (kStatsWarp<TPB>) {
     // the statistics warp's absmax of this thread's block
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s.stats[st], par))) {
@@ -352,10 +361,22 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
     if (lane == 0) mbar_arrive(&s.empty[st]);  // data is in registers: free the stage
 
     float m = amax;
+    if constexpr (PREW_T) {
+#pragma unroll
+      for (int j = 0; j < O::EPT; ++j) xe[j] = tile_elem<DT>(w, j);
+    }
+    (void)xe;
     if constexpr (TPB == 32) {
       // |x| >= 0 (or a NaN with the sign clear): the bits order as unsigned
       // integers, NaN above +inf, so one integer max reduces the warp
       m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+    } else if constexpr (TPB == 16) {
+      // the same integer reduction over each half-warp (the two halves are
+      // reduced one after the other, which for 2 groups still beats a 4-level
+      // shuffle tree: 1 GiB dyn8 bf16 blocksize 512 327.9 -> 313.6 us, fp32
+      // blocksize 256 225.7 -> 215.4 us; for 4 or more groups it did not)
+      const uint32_t gmask = 0xffffu << (lane & 16);
+      m = __uint_as_float(__reduce_max_sync(gmask, __float_as_uint(m)));
     } else if constexpr (TPB > 1) {
 #pragma unroll
       for (int off = 1; off < TPB; off <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -370,8 +391,8 @@ __device__ __forceinline__ bool quantize_tile(QSmem<E>& s, const QParams& p, uin
   constexpr bool kBucket = MODE == kModeLut || MODE == kModeLutF || MODE == kModeLutI;
   const bool fast = kBucket && (A == 0.0f || (A >= 0x1p-60f && A <= 0x1p60f));
   if (fast)
-    encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP>(
-        w, DT == kF32 ? make_scale_fast(A) : make_scale_fast_2term(A), t_base, ow);
+    encode_fast<DT, E, kBucket ? MODE : kModeLut, REMAP, PREW_T>(
+        w, DT == kF32 ? make_scale_fast(A) : make_scale_fast_2term(A), t_base, ow, xe);
   else encode_safe<DT, E, MODE>(w, make_scale(A), s.tab, s.lut, ow);
 
   const int64_t e0 = static_cast<int64_t>(tile) * TE + static_cast<int64_t>(ct) * O::EPT;
