@@ -64,17 +64,22 @@ N = 4 * 148 * 8 * 8192
 SKIP = 2 * 4 * 148
 
 
-def test_quantize_consumer_and_producer_waits_give_up(H):
+@pytest.mark.parametrize("bs,name", [(64, "nf4"), (4096, "nf4"), (4096, "dyn8")])
+def test_quantize_consumer_and_producer_waits_give_up(H, bs, name):
+    """Blocksize 64: the consumers' shuffle-tree form; blocksize 4096: the
+    statistics-warp forms (two statistics warps for NF4, one for dyn8),
+    whose statistics warps wait on the skipped tile as well."""
+    table = codebooks.get(name)
     x = synth.normal(N, "bf16", seed=31, std=0.02)
     xd = x.cuda()
-    code = torch.from_numpy(NF4).cuda()
-    a = torch.empty(N // 64, device="cuda")
-    q = torch.empty(N // 2, dtype=torch.uint8, device="cuda")
+    code = torch.from_numpy(table).cuda()
+    a = torch.empty(N // bs, device="cuda")
+    q = torch.empty(N // 2 if table.size == 16 else N, dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
     _fault(H, True)
     assert H.bq_test_skip_tile(SKIP) == bq.BQ_OK
     t0 = time.perf_counter()
-    assert H.bq_quantize_blockwise(xd.data_ptr(), bq.BQ_BF16, N, 64, code.data_ptr(), 16,
+    assert H.bq_quantize_blockwise(xd.data_ptr(), bq.BQ_BF16, N, bs, code.data_ptr(), table.size,
                                    a.data_ptr(), q.data_ptr(), 0) == bq.BQ_OK
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
@@ -86,11 +91,11 @@ def test_quantize_consumer_and_producer_waits_give_up(H):
     assert _fault(H, False) == 0, "reset did not clear the fault word"
     # the context is healthy: without the hook the same call gives the oracle's result
     assert H.bq_test_skip_tile(-1) == bq.BQ_OK
-    assert H.bq_quantize_blockwise(xd.data_ptr(), bq.BQ_BF16, N, 64, code.data_ptr(), 16,
+    assert H.bq_quantize_blockwise(xd.data_ptr(), bq.BQ_BF16, N, bs, code.data_ptr(), table.size,
                                    a.data_ptr(), q.data_ptr(), 0) == bq.BQ_OK
     torch.cuda.synchronize()
     assert _fault(H, True) == 0
-    oa, oq = oracle.quantize_blockwise_threaded(np_bits(x), "bf16", 64, NF4,
+    oa, oq = oracle.quantize_blockwise_threaded(np_bits(x), "bf16", bs, table,
                                                 oracle.host_threads())
     assert np.array_equal(a.cpu().numpy(), oa) and np.array_equal(q.cpu().numpy(), oq)
 
