@@ -521,9 +521,10 @@ def sweep_1gib(peak, reps=5, sample_blocks=1024):
     4096 elements from 2^28 on are zero, a whole block at every blocksize).
     Quantize, and dequantize to the input dtype, each timed with CUDA events
     (median of `reps` calls; the tensors exceed L2, so no flush).  A
-    stratified sample of each cell's blocks - every (nb // sample_blocks)-th
-    block, the zero block and the tail block - is compared bit for bit with
-    the oracle: absmax, codes and dequantized values."""
+    stratified sample of each cell's blocks - every (nfull // sample_blocks)-th
+    whole block, the zero block and the tail block (sample_check) - is
+    compared bit for bit with the oracle: absmax, codes and dequantized
+    values."""
     import dequantization_bq_quantize_b200 as bq
     import oracle
     dev = torch.device("cuda", torch.cuda.current_device())
