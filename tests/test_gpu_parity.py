@@ -743,33 +743,36 @@ def test_torch_helpers_check_option():
     bq.quantize_blockwise_host(x.cpu(), nf4, 64, chunk_elements=8192, check=True)
 
 
-def test_ring_stage_reuse_stress():
+@pytest.mark.parametrize("bs,name", [(64, "nf4"), (4096, "nf4"), (4096, "dyn8")])
+def test_ring_stage_reuse_stress(bs, name):
     """Thousands of quantize -> dequantize round trips of two alternating
-    inputs through the same buffers (a 14336 x 4096 bf16 matrix, NF4
-    blocksize 64), every output compared with references that are checked
-    against the oracle.  This catches a stage of a shared-memory ring being
-    refilled by its next bulk copy before every consumer has read it: before
-    the consumers' async-proxy fence, 16-warp dequantization CTAs gave a few
-    wrong warps per thousand round trips."""
-    nf4t = TABLES["nf4"]
-    nf4 = code_dev(nf4t)
+    inputs through the same buffers (a 14336 x 4096 bf16 matrix), every
+    output compared with references that are checked against the oracle.
+    This catches a stage of a shared-memory ring being refilled by its next
+    bulk copy before every consumer has read it: before the consumers'
+    async-proxy fence, 16-warp dequantization CTAs gave a few wrong warps per
+    thousand round trips.  Blocksize 4096 runs the statistics-warp forms of
+    the quantize kernel (their tamax slots are reused every four tiles) and,
+    for NF4, the streaming dequantization whose producer copies the scales."""
+    table = TABLES[name]
+    code = code_dev(table)
     n = 14336 * 4096
     xs, refs = [], []
     for seed in (1, 2):
         x = synth.normal(n, "bf16", seed=900 + seed, std=0.02)
-        oa, oq = oracle.quantize_blockwise_threaded(np_bits(x), "bf16", 64, nf4t, THREADS)
-        oy = oracle.dequantize_blockwise_threaded(oq, oa, n, 64, nf4t, "bf16", THREADS)
+        oa, oq = oracle.quantize_blockwise_threaded(np_bits(x), "bf16", bs, table, THREADS)
+        oy = oracle.dequantize_blockwise_threaded(oq, oa, n, bs, table, "bf16", THREADS)
         xs.append(x.cuda())
         refs.append((torch.from_numpy(oa).cuda(), torch.from_numpy(oq).cuda(),
                      torch.from_numpy(oy.view(np.int16)).cuda()))
-    a = torch.empty(n // 64, device="cuda")
-    q = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    a = torch.empty(n // bs, device="cuda")
+    q = torch.empty(n // 2 if table.size == 16 else n, dtype=torch.uint8, device="cuda")
     y = torch.empty(n, dtype=torch.bfloat16, device="cuda")
     bad = []
     for i in range(3000):
         k = i % 2
-        bq.quantize_blockwise(xs[k], nf4, 64, absmax=a, out=q)
-        bq.dequantize_blockwise(q, a, n, 64, nf4, out=y)
+        bq.quantize_blockwise(xs[k], code, bs, absmax=a, out=q)
+        bq.dequantize_blockwise(q, a, n, bs, code, out=y)
         ra, rq, ry = refs[k]
         if not (torch.equal(a, ra) and torch.equal(q, rq) and torch.equal(y.view(torch.int16), ry)):
             bad.append(i)
